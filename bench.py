@@ -1,0 +1,421 @@
+"""Benchmark of the KVarN hot path on B200: one JSON line on rank 0.
+
+A step is one pass of the whole path over one batch of the prefill-append
+workload (the one that names both halves): quantise-on-write of a 32768-token
+x 8-KV-head append batch (4096 K+V tiles, k4v2, 8 normalisation passes) into
+the paged cache, then one k4v2 decode-attention step for batch 8 at 16384
+context plus a ragged fp16 tail (Hq = 64, Hkv = 8, head_dim 128).  The rest of
+each sequence's 16K cache is quantised once before timing.
+
+  value  decode tokens/s of the whole step (B tokens per step, quantise
+         included), summed over ranks;
+  e2e    the same through the C-ABI with the step's inputs copied from pinned
+         host memory and the output read back inside the timed region.
+Per-kernel CUDA-event times give the quantise tiles/s, the decode-only
+tokens/s and each kernel's HBM GB/s from algorithmic bytes.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+--impl reference times the CPU oracle (the fp64 restatement in oracle/) on a
+bounded sample of the same step, extrapolated to the full step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "k4v2 decode attn tokens/s & HBM GB/s vs ~8 TB/s peak; quantize tiles/s"
+WORKLOAD = ("prefill-append + decode: quantize 32768 new tokens x 8 KV heads (4096 K+V tiles) into the paged "
+            "cache, then batch-8 decode at 16384 + ragged fp16 tail U{0..127}, Hq=64, Hkv=8, head_dim=128, "
+            "kvarn_k4v2_g128, 8 Sinkhorn iters")
+BATCH = 8
+HQ, HKV = 64, 8
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+# ------------------------------------------------------------------ clocks (NVML, sampled in a thread)
+
+class ClockSampler:
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._period = period_s
+        self._ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._ok = True
+        except Exception:
+            pass
+
+    def _run(self):
+        nv = self._nv
+        names = {0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+                 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, n in names.items():
+                    if r & bit:
+                        self.reasons.add(n)
+            except Exception:
+                pass
+            time.sleep(self._period)
+
+    def __enter__(self):
+        if self._ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ workload and byte counts
+
+def build_workload():
+    from bit_kv_cache_15_b200 import inputs
+    w, append_rows = inputs.prefill_append()
+    return w, append_rows
+
+
+def algorithmic_bytes(w, n_append_tokens):
+    """Bytes the path must move, per step (no workspace, no re-reads)."""
+    groups = n_append_tokens // 128
+    pairs = groups * HKV
+    q_bytes = pairs * ((32768 + 8192 + 528) + (32768 + 4096 + 528) + 2 * 8)   # in + codes + scales + slot
+    d_bytes = 0
+    for b in range(w.num_seqs):
+        L = int(w.seq_lens[b])
+        n_full, tl = L // 128, L % 128
+        d_bytes += HKV * (n_full * (12288 + 1056) + tl * 2 * 256 + n_full * 4)
+    d_bytes += 2 * w.num_seqs * HQ * 256                                             # q in, out
+    return q_bytes, d_bytes
+
+
+def traffic_record(kernel):
+    """DRAM bytes per launch from a committed ncu capture, if the kernel source is unchanged since."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    rec = json.load(open(p)).get(kernel)
+    if not rec:
+        return None
+    src = os.path.join(ROOT, "bit_kv_cache_15_b200", "csrc", rec["source"])
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    return rec["bytes_per_launch"] if sha == rec["source_sha"] else None
+
+
+# ------------------------------------------------------------------ our arm
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    from bit_kv_cache_15_b200 import kvarn as K
+
+    w, rows = build_workload()
+    cfg = K.config("kvarn_k4v2_g128")
+    packed, scales = K.alloc_cache(cfg, w.num_blocks, HKV, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    # one-time prefill of every full tile
+    K.quantize_tiles(torch.from_numpy(w.k_full).to(dev), torch.from_numpy(w.v_full).to(dev),
+                     torch.from_numpy(w.slot_mapping).to(dev), packed, scales, cfg, dev_status=status)
+    k_app = torch.from_numpy(np.ascontiguousarray(w.k_full[rows])).to(dev)
+    v_app = torch.from_numpy(np.ascontiguousarray(w.v_full[rows])).to(dev)
+    slot_app = torch.from_numpy(np.ascontiguousarray(w.slot_mapping[rows])).to(dev)
+    q = torch.from_numpy(w.q).to(dev)
+    tail = torch.from_numpy(w.tail).to(dev)
+    bt = torch.from_numpy(w.block_table).to(dev)
+    sl = torch.from_numpy(w.seq_lens).to(dev)
+    d = K.dims(BATCH, HQ, HKV, w.max_blocks_per_seq, w.num_blocks)
+    ws = torch.empty(K.decode_workspace_bytes(cfg, d), dtype=torch.uint8, device=dev)
+    out = torch.empty_like(q)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        K.quantize_tiles(k_app, v_app, slot_app, packed, scales, cfg, dev_status=status, stream=stream)
+        K.decode_attention(q, packed, scales, tail, bt, sl, cfg, out=out, workspace=ws, dev_status=status,
+                           stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0, "device status after warm-up"
+
+    # per-kernel event timing (separate pass, same work)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3 * args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        ev[3 * i].record(stream)
+        K.quantize_tiles(k_app, v_app, slot_app, packed, scales, cfg, dev_status=status, stream=stream)
+        ev[3 * i + 1].record(stream)
+        K.decode_attention(q, packed, scales, tail, bt, sl, cfg, out=out, workspace=ws, dev_status=status,
+                           stream=stream)
+        ev[3 * i + 2].record(stream)
+    torch.cuda.synchronize()
+    tq = [ev[3 * i].elapsed_time(ev[3 * i + 1]) for i in range(args.steps)]
+    td = [ev[3 * i + 1].elapsed_time(ev[3 * i + 2]) for i in range(args.steps)]
+
+    # the timed region: exactly K steps, barrier + sync on both sides
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with sampler:
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = e0.elapsed_time(e1)
+    assert int(status.item()) == 0, "device status after timing"
+
+    # end to end through the C-ABI: pinned host inputs in, output back, every step
+    h_k = torch.from_numpy(np.ascontiguousarray(w.k_full[rows])).pin_memory()
+    h_v = torch.from_numpy(np.ascontiguousarray(w.v_full[rows])).pin_memory()
+    h_slot = torch.from_numpy(np.ascontiguousarray(w.slot_mapping[rows])).pin_memory()
+    h_q = torch.from_numpy(w.q).pin_memory()
+    h_tail = torch.from_numpy(w.tail).pin_memory()
+    h_bt = torch.from_numpy(w.block_table).pin_memory()
+    h_sl = torch.from_numpy(w.seq_lens).pin_memory()
+    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (h_k, h_v, h_slot, h_q, h_tail, h_bt, h_sl))
+    d2h = h_out.numel() * h_out.element_size()
+
+    def e2e_step():
+        k_app.copy_(h_k, non_blocking=True)
+        v_app.copy_(h_v, non_blocking=True)
+        slot_app.copy_(h_slot, non_blocking=True)
+        q.copy_(h_q, non_blocking=True)
+        tail.copy_(h_tail, non_blocking=True)
+        bt.copy_(h_bt, non_blocking=True)
+        sl.copy_(h_sl, non_blocking=True)
+        step()
+        h_out.copy_(out, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    f1.record(stream)
+    torch.cuda.synchronize()
+    ms_e2e = f0.elapsed_time(f1)
+
+    if world > 1:
+        t = torch.tensor([ms, ms_e2e], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, ms_e2e = float(t[0]), float(t[1])
+
+    if rank == 0:
+        hbm_peak, peak_kind = load_peaks()
+        q_bytes, d_bytes = algorithmic_bytes(w, len(rows))
+        tq_ms, td_ms = statistics.median(tq), statistics.median(td)
+        q_gbs = q_bytes / (tq_ms * 1e-3) / 1e9
+        d_gbs = d_bytes / (td_ms * 1e-3) / 1e9
+        tiles = (len(rows) // 128) * HKV * 2
+        dominant = "quantize" if tq_ms >= td_ms else "decode"
+        dom_gbs, dom_ms = (q_gbs, tq_ms) if dominant == "quantize" else (d_gbs, td_ms)
+        traffic = traffic_record("quantize_kernel" if dominant == "quantize" else "decode_kernel")
+        clocks = sampler.summary()
+        line = {
+            "metric": METRIC,
+            "value": world * BATCH * args.steps / (ms * 1e-3),
+            "unit": "decode tokens/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": ms / args.steps,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "fp16 in/out, k4v2 codes, fp32 accumulate",
+            "data": "synthetic (seeded; Llama/Qwen-shaped GQA, outlier channels + lognormal token scales)",
+            "config": {"workload": WORKLOAD, "global_batch": BATCH * world, "seq_len": 16384,
+                       "parallelism": f"replicas x{world} (no collective on the path)",
+                       "l2": f"inputs larger than L2: {(q_bytes + d_bytes) / 1e6:.0f} MB of algorithmic traffic per step"},
+            "e2e": {"value": world * BATCH * args.steps / (ms_e2e * 1e-3), "unit": "decode tokens/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": 3 * args.steps,
+            "roofline": {"bound": "hbm", "kernel": dominant, "achieved": dom_gbs, "peak": hbm_peak,
+                         "unit": "GB/s", "frac": dom_gbs / hbm_peak, "traffic": traffic,
+                         "peak_kind": f"{peak_kind} (burst copy)"},
+            "kernels": {
+                "quantize": {"us": tq_ms * 1e3, "tiles_per_s": tiles / (tq_ms * 1e-3),
+                             "algorithmic_bytes": q_bytes, "hbm_gbs": q_gbs, "frac_of_measured_hbm": q_gbs / hbm_peak,
+                             "frac_of_8tbs": q_gbs / 8000.0},
+                "decode": {"us": td_ms * 1e3, "tokens_per_s": BATCH / (td_ms * 1e-3),
+                           "context_tokens_per_s": float(np.sum(w.seq_lens)) / (td_ms * 1e-3),
+                           "algorithmic_bytes": d_bytes, "hbm_gbs": d_gbs, "frac_of_measured_hbm": d_gbs / hbm_peak,
+                           "frac_of_8tbs": d_gbs / 8000.0},
+            },
+            "clocks": clocks,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(w, rows, budget_s=args.cpu_budget)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+# ------------------------------------------------------------------ the oracle (CPU baseline / reference arm)
+
+def oracle_step_sample(w, rows, n_tiles, n_pairs, seed=0):
+    """Time the oracle on n_tiles of the append batch and n_pairs (seq, KV head)
+    decodes (all G query heads), extrapolated to one full step."""
+    from oracle import kvarn_oracle as O
+    rng = np.random.default_rng(seed)
+    groups = len(rows) // 128
+    k_app, v_app = w.k_full[rows], w.v_full[rows]
+    t0 = time.perf_counter()
+    for _ in range(n_tiles):
+        g = int(rng.integers(groups))
+        h = int(rng.integers(HKV))
+        side = int(rng.integers(2))
+        src = k_app if side == 0 else v_app
+        O.quantize_tile(np.ascontiguousarray(src[g * 128:(g + 1) * 128, h]), 4 if side == 0 else 2, 8)
+    tq = time.perf_counter() - t0
+    # a small paged cache holding just the sampled pairs' tiles, quantised by the oracle (untimed)
+    G = HQ // HKV
+    t_dec = 0.0
+    for _ in range(n_pairs):
+        b = int(rng.integers(BATCH))
+        h = int(rng.integers(HKV))
+        s, e = w.token_range(b)
+        n_full = (e - s) // 128
+        sub_k = w.k_full[s:e, h:h + 1]
+        sub_v = w.v_full[s:e, h:h + 1]
+        slot = np.arange(e - s, dtype=np.int64)
+        packed, scales = O.quantize_tiles(sub_k, sub_v, slot, 1, n_full, 4, 2)
+        bt = np.arange(n_full, dtype=np.int32)[None, :]
+        q = w.q[b:b + 1, h * G:(h + 1) * G]
+        tail = w.tail[b:b + 1, :, h:h + 1]
+        t1 = time.perf_counter()
+        O.decode(q, packed, scales, tail, bt, w.seq_lens[b:b + 1], 1, 4, 2)
+        t_dec += time.perf_counter() - t1
+    tiles_total = groups * HKV * 2
+    pairs_total = BATCH * HKV
+    t_step = tq * tiles_total / max(n_tiles, 1) + t_dec * pairs_total / max(n_pairs, 1)
+    return t_step, tq + t_dec
+
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        return 1
+
+
+def cpu_baseline(w, rows, budget_s=20.0):
+    from threadpoolctl import threadpool_limits
+    with threadpool_limits(1):
+        t_step, spent = oracle_step_sample(w, rows, n_tiles=256, n_pairs=2)
+        reps = max(1, int(budget_s / max(spent, 1e-3)) - 1)
+        if reps > 1:
+            t_step2, spent2 = oracle_step_sample(w, rows, n_tiles=256 * reps, n_pairs=min(2 * reps, BATCH * HKV), seed=1)
+            t_step, spent = t_step2, spent + spent2
+    return {"value": BATCH / t_step, "unit": "decode tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"oracle (numpy fp64, 1 thread) on sampled append tiles and (seq, KV head) decodes of the "
+                      f"same step, extrapolated to 4096 tiles + 64 pairs; {spent:.1f} s of CPU work"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from threadpoolctl import threadpool_limits
+    w, rows = build_workload()
+    with threadpool_limits(1):
+        for i in range(args.warmup):
+            oracle_step_sample(w, rows, n_tiles=16, n_pairs=1, seed=100 + i)
+        t_steps, spent = [], 0.0
+        for i in range(args.steps):
+            t_step, s = oracle_step_sample(w, rows, n_tiles=32, n_pairs=1, seed=i)
+            t_steps.append(t_step)
+            spent += s
+    t_mean = float(np.mean(t_steps))
+    value = BATCH / t_mean
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "decode tokens/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_mean * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)", "data": "synthetic (seeded)",
+        "config": {"workload": WORKLOAD, "global_batch": BATCH, "seq_len": 16384, "parallelism": "none (CPU)"},
+        "cpu_baseline": {"value": value, "unit": "decode tokens/s", "cores": 1, "kind": "oracle",
+                         "sample": f"each step: 32 sampled append tiles + 1 (seq, KV head) decode, extrapolated to "
+                                   f"the full step; {spent:.1f} s of CPU work in total"},
+        "e2e": {"value": value, "unit": "decode tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

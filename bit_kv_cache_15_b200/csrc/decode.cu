@@ -1,0 +1,665 @@
+// decode.cu -- KVarN paged decode attention on the packed cache (sm_100a).
+//
+// Scales are folded in on read ([lehuy] "KVarN: Backend lượng tử hóa KV-cache
+// …", section Cơ chế hoạt động stage 4; [hypho] "KV-cache 量化终于能跑生产了？
+// KVarN …", section 它怎么做到的：四步流水线 step 4).  For sequence b, KV head
+// h and the G = Hq/Hkv query heads that read it, tile i with stored codes c,
+// log-scales Lt/Lc and grid zero/step contributes
+//   score_t = sm_scale/128 * 2^Lt_k[t] * (zero_k * sum_d q'_d + step_k * q'.c_t),
+//             q'_d = (q H)_d * 2^Lc_k[d]                       (key side)
+//   acc_d  += 2^Lc_v[d] * (zero_v * sum_t p'_t + step_v * sum_t p'_t c_td),
+//             p'_t = p_t * 2^Lt_v[t]                            (value side)
+// and the output is (acc H / 128 + tail part) / l.
+//
+// Grid: (num_splits + 1, Hkv, B), 4 warps per CTA.  CTA (s, h, b) with
+// s < num_splits owns tiles [s*T, s*T+T) of sequence b; its warps take them
+// round-robin, each warp running its own online softmax.  Each warp streams
+// its tiles through a private 2-stage shared-memory ring filled by bulk
+// copies (cp.async.bulk on the TMA engine).  Codes are laid out in the mma
+// fragment order, so a lane's 16-byte shared loads are its operands: a LOP3
+// turns each masked word into an f16x2 of exact small integers and one HFMA2
+// removes the magic offset.  Both contractions run on the tensor cores
+// (mma.m16n8k16, fp32 accumulate): K side rows = tokens, N = the 8 query
+// heads; V side rows = channels, N = heads, with the softmax weights moved
+// from accumulator to operand layout by movmatrix.  CTA s = num_splits
+// attends the fp16 tail (seq_len % 128 tokens) exactly, in the unrotated
+// domain.  A second kernel merges the partials and applies H / 128.
+#include <atomic>
+
+#include "common.cuh"
+#include "kvarn_internal.h"
+
+namespace kvarn {
+namespace {
+
+constexpr int kDWarps = 4;
+constexpr int kDThreads = 32 * kDWarps;
+constexpr int kDStages = 2;
+constexpr int kMaxG = 8;
+
+// A warp's work unit is 128/U tokens of one tile; U grows with the code size
+// so that 4 warps x 2 stages stay near 110 KB (two CTAs per SM).
+template <int KB, int VB>
+struct DecodeTraits {
+  static constexpr int kCodeK = 2048 * KB;
+  static constexpr int kCodeV = 2048 * VB;
+  static constexpr int kCode = kCodeK + kCodeV;
+  static constexpr int U = (KB + VB) <= 6 ? 1 : ((KB + VB) <= 12 ? 2 : 4);
+  static constexpr int MT = 8 / U;                    // 16-token blocks per unit
+  static constexpr int kUnitK = kCodeK / U;
+  static constexpr int kUnitV = kCodeV / U;
+  static constexpr int kStage = kUnitK + kUnitV + 2 * kScaleRec;
+  static constexpr int kBarOff = kDWarps * kDStages * kStage;
+  static constexpr int kQrotOff = kBarOff + 128;
+  static constexpr int kScrOff = kQrotOff + kMaxG * kHeadDim * 4;
+  static constexpr int kInvSigOff = kScrOff + kDWarps * kHeadDim * 4;
+  static constexpr int kSmem = kInvSigOff + 64;
+  static_assert(kStage % 16 == 0, "stage must stay 16-byte aligned");
+  static_assert(kSmem <= 227 * 1024, "shared memory");
+  static_assert(kDWarps * kDStages * 8 <= 128, "barrier area");
+};
+
+// f16x2 of the two codes in `slot` of a fragment-order word (low half-word:
+// even column, high half-word: odd column), as exact fp16 integers.
+template <int BITS>
+__device__ __forceinline__ uint32_t dequant_slot(uint32_t w, uint32_t w8, int slot) {
+  const int off = BITS * slot;
+  const int s = off & 7;
+  const uint32_t m1 = ((1u << BITS) - 1u) << s;
+  const uint32_t x = lop_and_or(off >= 8 ? w8 : w, m1 | (m1 << 16), 0x64006400u);
+  const uint32_t sc = static_cast<uint32_t>(15 - s) << 10;           // 2^-s
+  const uint32_t bi = 0x8000u | (static_cast<uint32_t>(25 - s) << 10);  // -1024 * 2^-s
+  return h2_as_u32(__hfma2(u32_as_h2(x), u32_as_h2(sc | (sc << 16)), u32_as_h2(bi | (bi << 16))));
+}
+
+__device__ __forceinline__ float hf(const __half* p, int i) { return __half2float(p[i]); }
+
+// ------------------------------------------------------------------ tail CTA
+
+__device__ void decode_tail(const DecodeArgs& p, uint8_t* smem, float* qs, int b, int h, int L) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tl = L & 127;
+  if (tl == 0) return;
+  const int G = p.G;
+  float* sc = reinterpret_cast<float*>(smem);  // [kMaxG][128] scores, then weights
+  for (int g = 0; g < kMaxG; ++g)
+    qs[g * 128 + tid] = g < G ? __half2float(p.q[((int64_t)b * p.Hq + h * G + g) * kHeadDim + tid]) : 0.f;
+  __syncthreads();
+  const float sl = p.sm_scale * kLog2e;
+  const __half* kt = p.tail + (((int64_t)b * 2 + 0) * p.Hkv + h) * (int64_t)(kTile * kHeadDim);
+  const __half* vt = p.tail + (((int64_t)b * 2 + 1) * p.Hkv + h) * (int64_t)(kTile * kHeadDim);
+  {
+    const int t = tid;
+    float dots[kMaxG];
+#pragma unroll
+    for (int g = 0; g < kMaxG; ++g) dots[g] = 0.f;
+    if (t < tl) {
+      const uint4* row = reinterpret_cast<const uint4*>(kt + (int64_t)t * kHeadDim);
+#pragma unroll 4
+      for (int c8 = 0; c8 < 16; ++c8) {
+        const uint4 raw = __ldg(row + c8);
+        const __half2* hp = reinterpret_cast<const __half2*>(&raw);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 kv = __half22float2(hp[i]);
+          const int d = c8 * 8 + 2 * i;
+#pragma unroll
+          for (int g = 0; g < kMaxG; ++g) dots[g] = fmaf(qs[g * 128 + d], kv.x, fmaf(qs[g * 128 + d + 1], kv.y, dots[g]));
+        }
+      }
+    }
+#pragma unroll
+    for (int g = 0; g < kMaxG; ++g) sc[g * 128 + t] = t < tl ? dots[g] * sl : -INFINITY;
+  }
+  __syncthreads();
+  __shared__ float mrow[kMaxG], lrow[kMaxG];
+  for (int g = warp; g < kMaxG; g += kDWarps) {
+    float v[4];
+    float m = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[i] = sc[g * 128 + lane + 32 * i];
+      m = fmaxf(m, v[i]);
+    }
+    m = warp_max(m);
+    float l = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float e = exp2f(v[i] - m);
+      sc[g * 128 + lane + 32 * i] = e;
+      l += e;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+    if (lane == 0) {
+      mrow[g] = m;
+      lrow[g] = l;
+    }
+  }
+  __syncthreads();
+  const int d = tid;
+  float acc[kMaxG];
+#pragma unroll
+  for (int g = 0; g < kMaxG; ++g) acc[g] = 0.f;
+  for (int t = 0; t < tl; ++t) {
+    const float vv = __half2float(vt[(int64_t)t * kHeadDim + d]);
+#pragma unroll
+    for (int g = 0; g < kMaxG; ++g) acc[g] = fmaf(sc[g * 128 + t], vv, acc[g]);
+  }
+  for (int g = 0; g < G; ++g) {
+    float* rec = p.ws + (((int64_t)b * p.Hq + h * G + g) * (p.num_splits + 1) + p.num_splits) * kPartialFloats;
+    if (d == 0) {
+      rec[0] = mrow[g];
+      rec[1] = lrow[g];
+      rec[2] = 0.f;
+      rec[3] = 0.f;
+    }
+    rec[4 + d] = acc[g];
+  }
+}
+
+// ------------------------------------------------------------------ main kernel
+
+template <int KB, int VB>
+__global__ void __launch_bounds__(kDThreads, 2) decode_kernel(const DecodeArgs p) {
+  using T = DecodeTraits<KB, VB>;
+  constexpr int U = T::U, MT = T::MT;
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + T::kBarOff);
+  float* qrot = reinterpret_cast<float*>(smem + T::kQrotOff);
+  float* invsig = reinterpret_cast<float*>(smem + T::kInvSigOff);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int G = p.G;
+  const int L = p.seq_lens[b];
+  if (L < 0 || L > kTile * p.max_blocks) {
+    if (tid == 0 && s == 0) report_status(p.status, KVARN_DEV_BAD_SEQ_LEN);
+    return;
+  }
+  if (s == p.num_splits) {
+    decode_tail(p, smem, qrot, b, h, L);
+    return;
+  }
+  const int n_full = L >> 7;
+  const int t_begin = s * p.tiles_per_split;
+  const int t_end = min(t_begin + p.tiles_per_split, n_full);
+  if (t_begin >= t_end) return;
+
+  if (tid == 0) {
+    for (int i = 0; i < kDWarps * kDStages; ++i) mbar_init(&bars[i], 1);
+    fence_barrier_init();
+  }
+
+  // ---- q H for the G heads, scaled by a power of two so |q H| <= 1 (a6)
+  {
+    const int g = tid >> 4, part = tid & 15;
+    float x[8];
+    if (g < G) {
+      const uint4 raw = __ldg(reinterpret_cast<const uint4*>(p.q + ((int64_t)b * p.Hq + h * G + g) * kHeadDim + part * 8));
+      const __half2* hp = reinterpret_cast<const __half2*>(&raw);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 f = __half22float2(hp[i]);
+        x[2 * i] = f.x;
+        x[2 * i + 1] = f.y;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) x[i] = 0.f;
+    }
+#pragma unroll
+    for (int hl = 1; hl < 8; hl <<= 1)
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        if ((i & hl) == 0) {
+          const float a = x[i], c = x[i + hl];
+          x[i] = a + c;
+          x[i + hl] = a - c;
+        }
+#pragma unroll
+    for (int m = 1; m < 16; m <<= 1) {
+      const bool up = (lane & m) != 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float y = __shfl_xor_sync(0xffffffffu, x[i], m);
+        x[i] = up ? (y - x[i]) : (x[i] + y);
+      }
+    }
+    float mx = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) mx = fmaxf(mx, fabsf(x[i]));
+#pragma unroll
+    for (int m = 1; m < 16; m <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, m));
+    int e = 0;
+    if (mx > 0.f) frexpf(mx, &e);
+    const float sig = ldexpf(1.f, -e);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) qrot[g * 128 + part * 8 + i] = x[i] * sig;
+    if (part == 0) invsig[g] = ldexpf(1.f, e);
+  }
+  __syncthreads();
+
+  // ---- per-warp state
+  const int g8 = lane >> 2, c = lane & 3;
+  float qr[32];   // q H of head g8 at channels 16kt + 2c + {0,1,8,9}
+#pragma unroll
+  for (int kt = 0; kt < 8; ++kt) {
+    const float2 lo = *reinterpret_cast<const float2*>(&qrot[g8 * 128 + 16 * kt + 2 * c]);
+    const float2 hi = *reinterpret_cast<const float2*>(&qrot[g8 * 128 + 16 * kt + 2 * c + 8]);
+    qr[4 * kt] = lo.x;
+    qr[4 * kt + 1] = lo.y;
+    qr[4 * kt + 2] = hi.x;
+    qr[4 * kt + 3] = hi.y;
+  }
+  const float coef0 = p.sm_scale * kLog2e * (1.f / 128.f) * invsig[2 * c];
+  const float coef1 = p.sm_scale * kLog2e * (1.f / 128.f) * invsig[2 * c + 1];
+  float* scr = reinterpret_cast<float*>(smem + T::kScrOff) + warp * kHeadDim;
+
+  float acc[8][4];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int r = 0; r < 4; ++r) acc[i][r] = 0.f;
+  float mrun[2] = {-INFINITY, -INFINITY}, lsum[2] = {0.f, 0.f};
+
+  // work units of this split: (tile, part), part in [0, U); warp takes every 4th
+  const int n_units = (t_end - t_begin) * U;
+  const int n_mine = warp < n_units ? (n_units - warp + kDWarps - 1) / kDWarps : 0;
+  uint8_t* stage_base = smem + warp * kDStages * T::kStage;
+  uint64_t* my_bars = bars + warp * kDStages;
+  const int32_t* btab = p.block_table + (int64_t)b * p.max_blocks;
+
+  // copy my k-th unit into stage k % 2; false for a bad block id
+  auto issue = [&](int k) {
+    const int unit = warp + k * kDWarps;
+    const int i = t_begin + unit / U, part = unit % U;
+    const int32_t blk = btab[i];
+    const bool ok = blk >= 0 && blk < p.num_blocks;
+    if (lane == 0) {
+      uint8_t* dst = stage_base + (k & 1) * T::kStage;
+      uint64_t* bar = &my_bars[k & 1];
+      if (ok) {
+        const uint8_t* cb = p.packed + ((int64_t)blk * p.Hkv + h) * T::kCode;
+        mbar_arrive_expect_tx(bar, T::kStage);
+        bulk_g2s(dst, cb + part * T::kUnitK, T::kUnitK, bar);
+        bulk_g2s(dst + T::kUnitK, cb + T::kCodeK + part * T::kUnitV, T::kUnitV, bar);
+        bulk_g2s(dst + T::kUnitK + T::kUnitV, p.scales + ((int64_t)blk * p.Hkv + h) * (2 * kScaleRec),
+                 2 * kScaleRec, bar);
+      } else {
+        report_status(p.status, KVARN_DEV_BAD_BLOCK);
+        mbar_arrive_expect_tx(bar, 0);   // completes the phase with no bytes
+      }
+    }
+    return ok;
+  };
+
+  bool ok0 = n_mine > 0 ? issue(0) : false;
+  bool ok1 = n_mine > 1 ? issue(1) : false;
+  int k_fail = -1;
+
+  for (int k = 0; k < n_mine; ++k) {
+    const int stg = k & 1;
+    if (!mbar_wait_bounded(&my_bars[stg], (k >> 1) & 1)) {
+      if (lane == 0) report_status(p.status, KVARN_DEV_TIMEOUT);
+      k_fail = k;
+      break;
+    }
+    const bool tile_ok = stg == 0 ? ok0 : ok1;
+    const int part = (warp + k * kDWarps) % U;
+    const uint8_t* st = stage_base + stg * T::kStage;
+    if (tile_ok) {
+      const uint8_t* rk = st + T::kUnitK + T::kUnitV;   // K scale record, V record follows
+      const __half* ltk = reinterpret_cast<const __half*>(rk);
+      const __half* lck = ltk + 128;
+      const float zk = *reinterpret_cast<const float*>(rk + 512);
+      const float sk = *reinterpret_cast<const float*>(rk + 516);
+      const __half* ltv = reinterpret_cast<const __half*>(rk + kScaleRec);
+      const __half* lcv = ltv + 128;
+      const float zv = *reinterpret_cast<const float*>(rk + kScaleRec + 512);
+      const float sv = *reinterpret_cast<const float*>(rk + kScaleRec + 516);
+      const int t0 = part * (16 * MT);   // first token of this unit within the tile
+
+      // a6: channel scales with a power-of-two prescale so q' <= 1 in magnitude
+      float lcl[4];
+      {
+        const float2 l01 = __half22float2(*reinterpret_cast<const __half2*>(lck + 4 * lane));
+        const float2 l23 = __half22float2(*reinterpret_cast<const __half2*>(lck + 4 * lane + 2));
+        lcl[0] = l01.x; lcl[1] = l01.y; lcl[2] = l23.x; lcl[3] = l23.y;
+      }
+      const float E = ceilf(warp_max(fmaxf(fmaxf(lcl[0], lcl[1]), fmaxf(lcl[2], lcl[3]))));
+      *reinterpret_cast<float4*>(&scr[4 * lane]) =
+          make_float4(exp2f(lcl[0] - E), exp2f(lcl[1] - E), exp2f(lcl[2] - E), exp2f(lcl[3] - E));
+      __syncwarp();
+      // q' as an fp16 hi + lo pair (about 22 significant bits): scores can reach
+      // |s| ~ 10 nats, where plain fp16 q' would cost ~1e-2 in the output
+      uint32_t qb0[8], qb1[8], ql0[8], ql1[8];
+      float qsum = 0.f;
+#pragma unroll
+      for (int kt = 0; kt < 8; ++kt) {
+        const float2 s01 = *reinterpret_cast<const float2*>(&scr[16 * kt + 2 * c]);
+        const float2 s89 = *reinterpret_cast<const float2*>(&scr[16 * kt + 2 * c + 8]);
+        const float x0 = qr[4 * kt] * s01.x, x1 = qr[4 * kt + 1] * s01.y;
+        const float x8 = qr[4 * kt + 2] * s89.x, x9 = qr[4 * kt + 3] * s89.y;
+        const __half2 h01 = __floats2half2_rn(x0, x1);
+        const __half2 h89 = __floats2half2_rn(x8, x9);
+        const float2 f01 = __half22float2(h01), f89 = __half22float2(h89);
+        const __half2 l01 = __floats2half2_rn(x0 - f01.x, x1 - f01.y);
+        const __half2 l89 = __floats2half2_rn(x8 - f89.x, x9 - f89.y);
+        const float2 g01 = __half22float2(l01), g89 = __half22float2(l89);
+        qb0[kt] = h2_as_u32(h01);
+        qb1[kt] = h2_as_u32(h89);
+        ql0[kt] = h2_as_u32(l01);
+        ql1[kt] = h2_as_u32(l89);
+        qsum += ((f01.x + g01.x) + (f01.y + g01.y)) + ((f89.x + g89.x) + (f89.y + g89.y));
+      }
+      __syncwarp();   // scr is rewritten by the next unit
+      qsum += __shfl_xor_sync(0xffffffffu, qsum, 1);
+      qsum += __shfl_xor_sync(0xffffffffu, qsum, 2);
+      const float qs0 = __shfl_sync(0xffffffffu, qsum, (2 * c) * 4);
+      const float qs1 = __shfl_sync(0xffffffffu, qsum, (2 * c + 1) * 4);
+      const float pw = ldexpf(1.f, static_cast<int>(E));
+      const float cf0 = coef0 * pw, cf1 = coef1 * pw;
+      const float za0 = zk * qs0, za1 = zk * qs1;
+
+      // a7: K-side contraction on the tensor cores (rows = this unit's tokens)
+      float S[MT][4];
+#pragma unroll
+      for (int i = 0; i < MT; ++i)
+#pragma unroll
+        for (int r = 0; r < 4; ++r) S[i][r] = 0.f;
+      {
+        constexpr int PK = 16 / KB;
+        uint32_t afr[4];
+#pragma unroll
+        for (int q = 0; q < 4 * KB / U; ++q) {
+          const uint4 v4 = *reinterpret_cast<const uint4*>(st + ((q * 32 + lane) << 4));
+          const uint32_t wds[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const uint32_t w = wds[i], w8 = w >> 8;
+#pragma unroll
+            for (int sl = 0; sl < PK; ++sl) {
+              const int rho = (4 * q + i) * PK + sl;
+              afr[rho & 3] = dequant_slot<KB>(w, w8, sl);
+              if ((rho & 3) == 3) {
+                const int blk = rho >> 2;   // (token block in unit) * 8 + channel block
+                mma_f16(S[blk >> 3], afr[0], afr[1], afr[2], afr[3], qb0[blk & 7], qb1[blk & 7]);
+                mma_f16(S[blk >> 3], afr[0], afr[1], afr[2], afr[3], ql0[blk & 7], ql1[blk & 7]);
+              }
+            }
+          }
+        }
+      }
+
+      // scores (log2 units) with the token scales, online softmax (a8)
+      float tv[MT][2];
+      float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+        for (int ri = 0; ri < 2; ++ri) {
+          const int t = t0 + 16 * mt + g8 + 8 * ri;
+          const float tk = exp2f(hf(ltk, t));
+          tv[mt][ri] = exp2f(hf(ltv, t));
+          S[mt][2 * ri] = fmaf(sk, S[mt][2 * ri], za0) * (cf0 * tk);
+          S[mt][2 * ri + 1] = fmaf(sk, S[mt][2 * ri + 1], za1) * (cf1 * tk);
+          mx0 = fmaxf(mx0, S[mt][2 * ri]);
+          mx1 = fmaxf(mx1, S[mt][2 * ri + 1]);
+        }
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+      }
+      const float mn0 = fmaxf(mrun[0], mx0), mn1 = fmaxf(mrun[1], mx1);
+      const float al0 = exp2f(mrun[0] - mn0), al1 = exp2f(mrun[1] - mn1);
+      mrun[0] = mn0;
+      mrun[1] = mn1;
+      float ls0 = 0.f, ls1 = 0.f, ps0 = 0.f, ps1 = 0.f;
+      uint32_t bv0[MT], bv1[MT];
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt) {
+        uint32_t pk[2];
+#pragma unroll
+        for (int ri = 0; ri < 2; ++ri) {
+          const float p0 = exp2f(S[mt][2 * ri] - mn0);
+          const float p1 = exp2f(S[mt][2 * ri + 1] - mn1);
+          ls0 += p0;
+          ls1 += p1;
+          const __half2 hp = __floats2half2_rn(p0 * tv[mt][ri], p1 * tv[mt][ri]);
+          const float2 fp = __half22float2(hp);
+          ps0 += fp.x;
+          ps1 += fp.y;
+          pk[ri] = h2_as_u32(hp);
+        }
+        bv0[mt] = movmatrix_t(pk[0]);
+        bv1[mt] = movmatrix_t(pk[1]);
+      }
+      lsum[0] = lsum[0] * al0 + ls0;
+      lsum[1] = lsum[1] * al1 + ls1;
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        ps0 += __shfl_xor_sync(0xffffffffu, ps0, o);
+        ps1 += __shfl_xor_sync(0xffffffffu, ps1, o);
+      }
+
+      // V-side contraction on the tensor cores (rows = channels, k = this unit's tokens)
+      float O[8][4];
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int r = 0; r < 4; ++r) O[i][r] = 0.f;
+      {
+        constexpr int PV = 16 / VB;
+        uint32_t afr[4];
+        const uint8_t* vc = st + T::kUnitK;
+#pragma unroll
+        for (int q = 0; q < 4 * VB / U; ++q) {
+          const uint4 v4 = *reinterpret_cast<const uint4*>(vc + ((q * 32 + lane) << 4));
+          const uint32_t wds[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const uint32_t w = wds[i], w8 = w >> 8;
+#pragma unroll
+            for (int sl = 0; sl < PV; ++sl) {
+              const int rho = (4 * q + i) * PV + sl;
+              afr[rho & 3] = dequant_slot<VB>(w, w8, sl);
+              if ((rho & 3) == 3) {
+                const int blk = rho >> 2;   // (token block in unit) * 8 + channel block
+                mma_f16(O[blk & 7], afr[0], afr[1], afr[2], afr[3], bv0[blk >> 3], bv1[blk >> 3]);
+              }
+            }
+          }
+        }
+      }
+
+      // fold the V grid and channel scales into the running accumulator
+      const float zp0 = zv * ps0, zp1 = zv * ps1;
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+        for (int ri = 0; ri < 2; ++ri) {
+          const float vcs = exp2f(hf(lcv, 16 * mt + g8 + 8 * ri));
+          acc[mt][2 * ri] = fmaf(acc[mt][2 * ri], al0, vcs * fmaf(sv, O[mt][2 * ri], zp0));
+          acc[mt][2 * ri + 1] = fmaf(acc[mt][2 * ri + 1], al1, vcs * fmaf(sv, O[mt][2 * ri + 1], zp1));
+        }
+    }
+    __syncwarp();
+    if (k + 2 < n_mine) {
+      const bool okn = issue(k + 2);
+      if (stg == 0) ok0 = okn; else ok1 = okn;
+    }
+  }
+
+  if (k_fail >= 0) {
+    // let the copies still in flight land before this CTA's shared memory is released
+    (void)mbar_wait_bounded(&my_bars[k_fail & 1], (k_fail >> 1) & 1);
+    if (k_fail + 1 < n_mine) (void)mbar_wait_bounded(&my_bars[(k_fail + 1) & 1], ((k_fail + 1) >> 1) & 1);
+  }
+
+  // ---- merge the four warps and write the partial (m, l, acc) per head
+#pragma unroll
+  for (int o = 4; o < 32; o <<= 1) {
+    lsum[0] += __shfl_xor_sync(0xffffffffu, lsum[0], o);
+    lsum[1] += __shfl_xor_sync(0xffffffffu, lsum[1], o);
+  }
+  __syncthreads();   // all warps are done with their stages
+  float* mS = reinterpret_cast<float*>(smem);            // [4][8]
+  float* lS = mS + kDWarps * kMaxG;                      // [4][8]
+  float* aS = lS + kDWarps * kMaxG;                      // [4][8][128]
+  if (g8 == 0) {
+    mS[warp * kMaxG + 2 * c] = mrun[0];
+    mS[warp * kMaxG + 2 * c + 1] = mrun[1];
+    lS[warp * kMaxG + 2 * c] = lsum[0];
+    lS[warp * kMaxG + 2 * c + 1] = lsum[1];
+  }
+#pragma unroll
+  for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+    for (int ri = 0; ri < 2; ++ri) {
+      const int d = 16 * mt + g8 + 8 * ri;
+      aS[(warp * kMaxG + 2 * c) * kHeadDim + d] = acc[mt][2 * ri];
+      aS[(warp * kMaxG + 2 * c + 1) * kHeadDim + d] = acc[mt][2 * ri + 1];
+    }
+  __syncthreads();
+  const int d = tid;
+  for (int g = 0; g < G; ++g) {
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kDWarps; ++w) M = fmaxf(M, mS[w * kMaxG + g]);
+    float l = 0.f, a = 0.f;
+#pragma unroll
+    for (int w = 0; w < kDWarps; ++w) {
+      const float mw = mS[w * kMaxG + g];
+      const float f = mw == -INFINITY ? 0.f : exp2f(mw - M);
+      l = fmaf(f, lS[w * kMaxG + g], l);
+      a = fmaf(f, aS[(w * kMaxG + g) * kHeadDim + d], a);
+    }
+    float* rec = p.ws + (((int64_t)b * p.Hq + h * G + g) * (p.num_splits + 1) + s) * kPartialFloats;
+    if (d == 0) {
+      rec[0] = M;
+      rec[1] = l;
+      rec[2] = 0.f;
+      rec[3] = 0.f;
+    }
+    rec[4 + d] = a;
+  }
+}
+
+// ------------------------------------------------------------------ combine (a10)
+
+__global__ void __launch_bounds__(128) combine_kernel(const DecodeArgs p) {
+  const int wg = blockIdx.x * 4 + (threadIdx.x >> 5);
+  if (wg >= p.B * p.Hq) return;
+  const int lane = threadIdx.x & 31;
+  const int b = wg / p.Hq, j = wg % p.Hq;
+  int L = p.seq_lens[b];
+  __half* o = p.out + ((int64_t)b * p.Hq + j) * kHeadDim + 4 * lane;
+  if (L <= 0 || L > kTile * p.max_blocks) {
+    *reinterpret_cast<uint2*>(o) = make_uint2(0u, 0u);
+    return;
+  }
+  const int n_full = L >> 7;
+  const int nsv = (n_full + p.tiles_per_split - 1) / p.tiles_per_split;
+  const bool has_tail = (L & 127) != 0;
+  const float* rec = p.ws + ((int64_t)b * p.Hq + j) * (p.num_splits + 1) * kPartialFloats;
+  const float* trec = rec + (int64_t)p.num_splits * kPartialFloats;
+  float M = has_tail ? trec[0] : -INFINITY;
+  for (int s = 0; s < nsv; ++s) M = fmaxf(M, rec[(int64_t)s * kPartialFloats]);
+  float l = 0.f, a[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int s = 0; s < nsv; ++s) {
+    const float* r = rec + (int64_t)s * kPartialFloats;
+    const float w = exp2f(r[0] - M);
+    l = fmaf(w, r[1], l);
+    const float4 v = *reinterpret_cast<const float4*>(r + 4 + 4 * lane);
+    a[0] = fmaf(w, v.x, a[0]);
+    a[1] = fmaf(w, v.y, a[1]);
+    a[2] = fmaf(w, v.z, a[2]);
+    a[3] = fmaf(w, v.w, a[3]);
+  }
+  // acc H / 128: channels 4*lane .. 4*lane+3 in this lane
+  {
+    float b0 = a[0] + a[1], b1 = a[0] - a[1], b2 = a[2] + a[3], b3 = a[2] - a[3];
+    a[0] = b0 + b2; a[1] = b1 + b3; a[2] = b0 - b2; a[3] = b1 - b3;
+#pragma unroll
+    for (int m = 1; m < 32; m <<= 1) {
+      const bool up = (lane & m) != 0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float y = __shfl_xor_sync(0xffffffffu, a[i], m);
+        a[i] = up ? (y - a[i]) : (a[i] + y);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) a[i] *= (1.f / 128.f);
+  }
+  if (has_tail) {
+    const float w = exp2f(trec[0] - M);
+    l = fmaf(w, trec[1], l);
+    const float4 v = *reinterpret_cast<const float4*>(trec + 4 + 4 * lane);
+    a[0] = fmaf(w, v.x, a[0]);
+    a[1] = fmaf(w, v.y, a[1]);
+    a[2] = fmaf(w, v.z, a[2]);
+    a[3] = fmaf(w, v.w, a[3]);
+  }
+  const float il = 1.f / l;
+  const __half2 o01 = __floats2half2_rn(a[0] * il, a[1] * il);
+  const __half2 o23 = __floats2half2_rn(a[2] * il, a[3] * il);
+  *reinterpret_cast<uint2*>(o) = make_uint2(h2_as_u32(o01), h2_as_u32(o23));
+}
+
+template <int KB, int VB>
+cudaError_t launch_d(const DecodeArgs& p, cudaStream_t stream) {
+  using T = DecodeTraits<KB, VB>;
+  static std::atomic<uint64_t> configured{0};   // one bit per device ordinal
+  int dev = 0;
+  cudaError_t e0 = cudaGetDevice(&dev);
+  if (e0 != cudaSuccess) return e0;
+  const uint64_t bit = 1ull << (dev & 63);
+  if ((configured.load(std::memory_order_acquire) & bit) == 0) {
+    cudaError_t e = cudaFuncSetAttribute(decode_kernel<KB, VB>, cudaFuncAttributeMaxDynamicSharedMemorySize, T::kSmem);
+    if (e != cudaSuccess) return e;
+    configured.fetch_or(bit, std::memory_order_acq_rel);
+  }
+  const dim3 grid(static_cast<unsigned>(p.num_splits + 1), static_cast<unsigned>(p.Hkv), static_cast<unsigned>(p.B));
+  decode_kernel<KB, VB><<<grid, kDThreads, T::kSmem, stream>>>(p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const unsigned nc = static_cast<unsigned>((p.B * p.Hq + 3) / 4);
+  combine_kernel<<<nc, 128, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+void decode_geometry(int B, int Hkv, int max_blocks, int* tiles_per_split, int* num_splits) {
+  // Aim at about two resident CTAs per SM on a 148-SM part, four tiles per CTA at least.
+  const int pairs = B * Hkv > 0 ? B * Hkv : 1;
+  const int target = 2 * 148 * 2;
+  const int want = (target + pairs - 1) / pairs;
+  int T = (max_blocks + want - 1) / want;
+  if (T < kDWarps) T = kDWarps;
+  int ns = (max_blocks + T - 1) / T;
+  if (ns < 1) ns = 1;
+  *tiles_per_split = T;
+  *num_splits = ns;
+}
+
+cudaError_t launch_decode(const DecodeArgs& p, cudaStream_t stream) {
+#define KVARN_D_CASE(KB, VB) \
+  if (p.kb == KB && p.vb == VB) return launch_d<KB, VB>(p, stream);
+  KVARN_D_CASE(4, 2)
+  KVARN_D_CASE(2, 2)
+  KVARN_D_CASE(4, 4)
+  KVARN_D_CASE(8, 8)
+  KVARN_D_CASE(2, 4)
+  KVARN_D_CASE(4, 8)
+  KVARN_D_CASE(8, 4)
+  KVARN_D_CASE(8, 2)
+  KVARN_D_CASE(2, 8)
+#undef KVARN_D_CASE
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace kvarn

@@ -1,0 +1,69 @@
+// kvarn_internal.h -- launch descriptors shared by the host layer and the kernels.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace kvarn {
+
+struct QuantArgs {
+  const __half* k;
+  const __half* v;
+  const int64_t* slot_mapping;
+  int64_t num_groups;   // num_tokens / 128
+  int hkv;
+  int64_t num_blocks;
+  uint8_t* packed;
+  uint8_t* scales;
+  int iters;
+  int kb, vb;
+  float* dbg;           // nullable: fp32 log-scales before rounding
+  int32_t* status;      // nullable
+};
+
+// One split-K partial record: m, l, two pad words, acc[128]  (528 bytes).
+constexpr int kPartialFloats = 132;
+
+struct DecodeArgs {
+  const __half* q;
+  const uint8_t* packed;
+  const uint8_t* scales;
+  const __half* tail;
+  const int32_t* block_table;
+  const int32_t* seq_lens;
+  __half* out;
+  float* ws;
+  int B, Hq, Hkv, G, max_blocks;
+  int64_t num_blocks;
+  int kb, vb;
+  int tiles_per_split, num_splits;
+  float sm_scale;
+  int32_t* status;
+};
+
+// Split-K geometry: a pure function of the dims (never of seq_lens).
+void decode_geometry(int B, int Hkv, int max_blocks, int* tiles_per_split, int* num_splits);
+
+cudaError_t launch_quantize(const QuantArgs& p, cudaStream_t stream);
+cudaError_t launch_decode(const DecodeArgs& p, cudaStream_t stream);
+
+struct BaselineArgs {
+  const __half* q;
+  const void* k_cache;
+  const void* v_cache;
+  const int32_t* block_table;
+  const int32_t* seq_lens;
+  __half* out;
+  float* ws;
+  int B, Hq, Hkv, G, max_blocks;
+  int64_t num_blocks;
+  int tiles_per_split, num_splits;
+  float sm_scale, k_scale, v_scale;
+  int fp8;               // 0 = fp16 cache, 1 = e4m3 cache
+  int32_t* status;
+};
+
+cudaError_t launch_baseline(const BaselineArgs& p, cudaStream_t stream);
+
+}  // namespace kvarn

@@ -1,0 +1,289 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
+
+Quantizer, staged as in the tolerance plan:
+  1. fp32 log-scales before rounding: the scale 2^lt within 1e-5 relative,
+     i.e. |lt_gpu - lt_oracle| <= log2(1 + 1e-5);
+  2. stored fp16 log-scales: the fp16 rounding of some value within that
+     tolerance of the oracle's fp64 value (at a rounding boundary either
+     neighbour is correct);
+  3. codes re-derived by the oracle (fp32, its own exact rotation) from the
+     GPU's stored scales, zero and step: every mismatch is +-1 at a rounding
+     tie, within the fp32 error bound of the GPU's rotation;
+  4. end-to-end codes >= 99.99 % identical to the oracle's own.
+Decode: <= 2e-3 absolute (one fp16 step where |o| >= 4 makes that step
+larger) against the oracle's explicit-dequant attention over the GPU's own
+packed cache (read through the oracle's own unpacker).
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import kvarn_oracle as O
+from bit_kv_cache_15_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+DECODE_TOL = 2e-3
+
+
+@pytest.fixture(scope="module")
+def K():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from bit_kv_cache_15_b200 import build
+    build.build()
+    from bit_kv_cache_15_b200 import kvarn
+    return kvarn
+
+
+def _dev(x, dtype=None):
+    t = torch.from_numpy(np.ascontiguousarray(x))
+    if dtype is not None:
+        t = t.to(dtype)
+    return t.cuda()
+
+
+def gpu_quantize(K, k, v, slot, num_blocks, cfg_str="kvarn_k4v2_g128", debug=True):
+    cfg = K.config(cfg_str)
+    hkv = k.shape[1]
+    packed, scales = K.alloc_cache(cfg, num_blocks, hkv)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    dbg = torch.zeros((k.shape[0] // 128, hkv, 2, 256), dtype=torch.float32, device="cuda") if debug else None
+    K.quantize_tiles(_dev(k), _dev(v), _dev(slot), packed, scales, cfg, dev_status=status, debug_logscales=dbg)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    return (packed.cpu().numpy(), scales.cpu().numpy(), dbg.cpu().numpy() if debug else None)
+
+
+# "scales within 1e-5 relative": the scale factor is 2^lt, so the log-scale
+# may differ by log2(1 + 1e-5)
+LOG_TOL = float(np.log2(1.0 + 1e-5))
+
+
+def _fp16_neighbours_ok(gpu16, x64, tol=LOG_TOL):
+    """gpu16 is the fp16 rounding of some value within tol of the oracle's
+    fp64 x64 (either neighbour is correct at a rounding boundary); rounding
+    is monotone, so that is the interval [fp16(x - tol), fp16(x + tol)]."""
+    lo = (x64 - tol).astype(np.float16).astype(np.float64)
+    hi = (x64 + tol).astype(np.float16).astype(np.float64)
+    g = gpu16.astype(np.float64)
+    return (g >= lo) & (g <= hi)
+
+
+def check_quantize_parity(K, k, v, slot, num_blocks, kb, vb, groups=None, report=None):
+    packed, scales, dbg = gpu_quantize(K, k, v, slot, num_blocks, f"kvarn_k{kb}v{vb}_g128")
+    hkv = k.shape[1]
+    n_groups = k.shape[0] // 128
+    groups = range(n_groups) if groups is None else groups
+    total = mism_e2e = mism_given = 0
+    worst_scale = 0.0
+    for g in groups:
+        blk = int(slot[g * 128]) // 128
+        for h in range(hkv):
+            for side, src, bits in (("K", k, kb), ("V", v, vb)):
+                x = np.ascontiguousarray(src[g * 128:(g + 1) * 128, h, :])
+                r = O.quantize_tile(x, bits, 8)
+                codes, Lt, Lc, zero, step = O.read_tile(packed, scales, blk, h, side, kb, vb)
+                sidx = 0 if side == "K" else 1
+                lt_gpu = dbg[g, h, sidx, :128].astype(np.float64)
+                lc_gpu = dbg[g, h, sidx, 128:].astype(np.float64)
+                # stage 1
+                e1 = np.max(np.abs(lt_gpu - r["lt"]))
+                e2 = np.max(np.abs(lc_gpu - r["lc"]))
+                worst_scale = max(worst_scale, e1, e2)
+                assert e1 <= LOG_TOL and e2 <= LOG_TOL, (g, h, side, e1, e2)
+                # stage 2
+                assert np.all(_fp16_neighbours_ok(Lt, r["lt"])), (g, h, side)
+                assert np.all(_fp16_neighbours_ok(Lc, r["lc"])), (g, h, side)
+                # stage 3: codes given the GPU's stored scales, zero and step
+                R32 = r["R"].astype(np.float32)
+                c_given, z2, s2, y = O.quantize_given_scales(R32, Lt, Lc, bits)
+                assert abs(float(z2) - float(zero)) <= 1e-6 * max(1.0, abs(float(zero))) + 1e-30, (z2, zero)
+                assert abs(float(s2) - float(step)) <= 1e-6 * float(s2), (s2, step)
+                c_g, _, _, y_g = O.quantize_given_scales(R32, Lt, Lc, bits, zero, step)
+                diff = codes != c_g
+                if diff.any():
+                    assert np.all(np.abs(codes[diff] - c_g[diff]) == 1)
+                    mt = O.multipliers(Lt).astype(np.float64)[:, None]
+                    mc = O.multipliers(Lc).astype(np.float64)[None, :]
+                    dR = 2.0 ** -18 * np.abs(x.astype(np.float64)).sum(axis=1)[:, None]
+                    dy = dR * mt * mc / float(step) + 2.0 ** -20 * np.abs(y_g)
+                    frac = np.abs(y_g - np.floor(y_g) - 0.5)
+                    assert np.all(frac[diff] <= dy[diff]), (g, h, side, frac[diff].max())
+                mism_given += int(diff.sum())
+                # stage 4
+                mism_e2e += int((codes != r["codes"]).sum())
+                total += codes.size
+    if report is not None:
+        report.update(total=total, mism_e2e=mism_e2e, mism_given=mism_given, worst_scale=worst_scale)
+    assert mism_e2e <= 1e-4 * total, (mism_e2e, total)
+    return packed, scales
+
+
+@pytest.mark.parametrize("kb,vb", [(4, 2), (2, 2), (4, 4), (8, 8)])
+def test_quantize_parity_small(K, kb, vb):
+    """24 token groups x 2 heads x {K,V} = 96 tiles, shuffled slots."""
+    prob = inputs.quantize_batch(seed=7 + kb * 10 + vb, num_tokens=128 * 24, num_kv_heads=2, num_blocks=40)
+    rep = {}
+    check_quantize_parity(K, prob["k"], prob["v"], prob["slot_mapping"], prob["num_blocks"], kb, vb, report=rep)
+    print(f"k{kb}v{vb}: {rep}")
+
+
+def test_quantize_tiny_and_special_tiles(K):
+    """The tiny workload, a zero tile and a rank-one tile."""
+    w = inputs.tiny()
+    check_quantize_parity(K, w.k_full, w.v_full, w.slot_mapping, w.num_blocks, 4, 2)
+    z = np.zeros((128, 1, 128), np.float16)
+    packed, scales, _ = gpu_quantize(K, z, z, np.arange(128, dtype=np.int64), 1)
+    codes, Lt, Lc, zero, step = O.read_tile(packed, scales, 0, 0, "K", 4, 2)
+    assert np.all(codes == 0) and step == 1.0 and np.all(np.isfinite(Lt.astype(np.float32)))
+
+
+def test_quantize_status_on_bad_slot(K):
+    cfg = K.config()
+    k = torch.zeros((256, 1, 128), dtype=torch.float16, device="cuda")
+    packed, scales = K.alloc_cache(cfg, 2, 1)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    slot = torch.tensor(list(range(128)) + [5 * 128 + i for i in range(128)], dtype=torch.int64, device="cuda")
+    K.quantize_tiles(k, k, slot, packed, scales, cfg, dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 1          # block 5 is beyond a 2-block pool
+    status.zero_()
+    slot[128:] = torch.arange(128, device="cuda") + 7   # misaligned start
+    K.quantize_tiles(k, k, slot, packed, scales, cfg, dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 1
+
+
+# ------------------------------------------------------------------ decode
+
+def run_decode(K, w, kb=4, vb=2, packed=None, scales=None):
+    cfg = K.config(f"kvarn_k{kb}v{vb}_g128")
+    if packed is None:
+        packed, scales = K.alloc_cache(cfg, w.num_blocks, w.num_kv_heads)
+        if w.k_full.shape[0]:
+            K.quantize_tiles(_dev(w.k_full), _dev(w.v_full), _dev(w.slot_mapping), packed, scales, cfg)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = K.decode_attention(_dev(w.q), packed, scales, _dev(w.tail), _dev(w.block_table), _dev(w.seq_lens), cfg,
+                             dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    return out.cpu().numpy(), packed.cpu().numpy(), scales.cpu().numpy()
+
+
+def decode_bound(ref16):
+    """2e-3 absolute, or one fp16 step where the output's own spacing is
+    larger (|o| >= 4): two fp16 results cannot be closer than one step
+    unless they are equal."""
+    r = np.abs(ref16.astype(np.float16))
+    step = np.spacing(r).astype(np.float64)
+    return np.maximum(DECODE_TOL, step)
+
+
+def decode_errors(out, ref, pairs):
+    err = np.zeros(0)
+    bnd = np.zeros(0)
+    mag = np.zeros(0)
+    for b, j in pairs:
+        e = np.abs(out[b, j].astype(np.float64) - ref[b, j].astype(np.float64))
+        err = np.concatenate([err, e])
+        bnd = np.concatenate([bnd, decode_bound(ref[b, j])])
+        mag = np.concatenate([mag, np.abs(ref[b, j].astype(np.float64))])
+    return err, bnd, mag
+
+
+def check_decode(K, w, kb=4, vb=2, heads=None):
+    out, packed, scales = run_decode(K, w, kb, vb)
+    ref = O.decode(w.q, packed, scales, w.tail, w.block_table, w.seq_lens, w.num_kv_heads, kb, vb, heads=heads)
+    pairs = heads if heads is not None else [(b, j) for b in range(w.num_seqs) for j in range(w.num_q_heads)]
+    err, bnd, mag = decode_errors(out, ref, pairs)
+    small = mag < 4
+    print(f"decode max err {err.max():.2e} (|o|<4: {err[small].max() if small.any() else 0:.2e}, "
+          f"|o|>=4: {err[~small].max() if (~small).any() else 0:.2e}, n>=4: {(~small).sum()})")
+    assert np.all(err <= bnd), float(np.max(err - bnd))
+    return float(err.max()), out
+
+
+@pytest.mark.parametrize("G", [1, 4, 8])
+def test_decode_parity_ragged(K, G):
+    """Tail-only, exactly one tile, tile + tail, many tiles (several splits), empty."""
+    lens = [77, 128, 300, 40 * 128 + 5, 0, 129, 1]
+    w = inputs.make_decode_workload("ragged", lens, 2 * G, 2, seed=300 + G, pool_blocks=80)
+    err, out = check_decode(K, w)
+    assert np.all(out[4] == 0)                      # empty sequence
+    print(f"G={G} max abs err {err:.2e}")
+
+
+@pytest.mark.parametrize("kb,vb", [(2, 2), (4, 4), (8, 8), (2, 4), (8, 2)])
+def test_decode_parity_precisions(K, kb, vb):
+    w = inputs.make_decode_workload("prec", [20 * 128 + 33, 3 * 128], 16, 2, seed=400 + kb * 10 + vb)
+    err, _ = check_decode(K, w, kb, vb)
+    print(f"k{kb}v{vb} max abs err {err:.2e}")
+
+
+def test_decode_tiny(K):
+    err, _ = check_decode(K, inputs.tiny())
+    print(f"tiny max abs err {err:.2e}")
+
+
+def test_decode_status_codes(K):
+    w = inputs.make_decode_workload("st", [256, 300], 4, 1, seed=9, pool_blocks=4)
+    cfg = K.config()
+    packed, scales = K.alloc_cache(cfg, w.num_blocks, 1)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    bt = w.block_table.copy()
+    bt[1, 1] = 99                                   # beyond the 4-block pool
+    K.decode_attention(_dev(w.q), packed, scales, _dev(w.tail), _dev(bt), _dev(w.seq_lens), cfg, dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 2
+    status.zero_()
+    sl = w.seq_lens.copy()
+    sl[0] = 128 * w.max_blocks_per_seq + 1          # longer than the block table
+    K.decode_attention(_dev(w.q), packed, scales, _dev(w.tail), _dev(w.block_table), _dev(sl), cfg, dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 3
+
+
+def test_decode_quality_vs_fp16_reported(K):
+    """Reported, not gated: k4v2 decode against fp16 attention on the unquantised cache."""
+    w = inputs.make_decode_workload("q", [16 * 128 + 50] * 2, 16, 2, seed=11)
+    out, _, _ = run_decode(K, w)
+    rows_k, rows_v = [], []
+    for b in range(2):
+        s, e = w.token_range(b)
+        tl = int(w.seq_lens[b]) % 128
+        rows_k.append(np.concatenate([w.k_full[s:e], w.tail[b, 0, :, :tl].transpose(1, 0, 2)]))
+        rows_v.append(np.concatenate([w.v_full[s:e], w.tail[b, 1, :, :tl].transpose(1, 0, 2)]))
+    ref = O.decode_uncompressed(w.q, rows_k, rows_v, w.seq_lens, 2).astype(np.float64)
+    rel = np.abs(out.astype(np.float64) - ref).mean() / np.abs(ref).mean()
+    print(f"k4v2 vs fp16 attention: mean relative error {rel:.3f}")
+    assert rel < 1.0
+
+
+# ------------------------------------------------------------------ full-size, sampled
+
+def test_full_size_qwen3_32b_sampled(K):
+    """The Qwen3-32B-shaped workload (B=8, 16K + ragged tail, 64/8 heads) in the
+    bench's launch configuration: all tiles quantised and decoded on the GPU,
+    a sample of tiles and outputs checked against the oracle."""
+    w = inputs.qwen3_32b()
+    cfg = K.config()
+    packed, scales = K.alloc_cache(cfg, w.num_blocks, w.num_kv_heads)
+    dbg = torch.zeros((w.k_full.shape[0] // 128, 8, 2, 256), dtype=torch.float32, device="cuda")
+    K.quantize_tiles(_dev(w.k_full), _dev(w.v_full), _dev(w.slot_mapping), packed, scales, cfg, debug_logscales=dbg)
+    out, packed_h, scales_h = run_decode(K, w, packed=packed, scales=scales)
+    rng = np.random.default_rng(5)
+    n_groups = w.k_full.shape[0] // 128
+    for g in rng.choice(n_groups, size=6, replace=False):
+        blk = int(w.slot_mapping[g * 128]) // 128
+        for h in (0, 5):
+            for side, src, bits in (("K", w.k_full, 4), ("V", w.v_full, 2)):
+                r = O.quantize_tile(np.ascontiguousarray(src[g * 128:(g + 1) * 128, h]), bits, 8)
+                codes, Lt, Lc, z, s = O.read_tile(packed_h, scales_h, blk, h, side, 4, 2)
+                assert (codes != r["codes"]).mean() <= 1e-3
+                assert np.all(_fp16_neighbours_ok(Lt, r["lt"]))
+    heads = [(0, 0), (3, 17), (7, 63)]
+    ref = O.decode(w.q, packed_h, scales_h, w.tail, w.block_table, w.seq_lens, 8, 4, 2, heads=heads)
+    err, bnd, _ = decode_errors(out, ref, heads)
+    assert np.all(err <= bnd)
+    assert np.all(np.isfinite(out.astype(np.float32)))
