@@ -25,6 +25,7 @@
 // attends the fp16 tail (seq_len % 128 tokens) exactly, in the unrotated
 // domain.  A second kernel merges the partials and applies H / 128.
 #include <atomic>
+#include <mutex>
 
 #include "common.cuh"
 #include "kvarn_internal.h"
@@ -632,6 +633,32 @@ cudaError_t launch_d(const DecodeArgs& p, cudaStream_t stream) {
 }
 
 }  // namespace
+
+// ------------------------------------------------------------------ fixed scratch
+// Device-resident scratch for kvarn_decode_attention_noalloc: the split-K
+// partial records live in this file-scope array instead of a caller-supplied
+// workspace.  Every GPU that loads the library holds these bytes until exit.
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchBytes / sizeof(float)];
+
+cudaError_t noalloc_scratch(void** ptr, size_t* bytes) {
+  static std::mutex mu;
+  static void* addr[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    // once per device, with that device current: the symbol's device address
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    addr[dev] = p;
+  }
+  *ptr = addr[dev];
+  *bytes = kNoAllocScratchBytes;
+  return cudaSuccess;
+}
 
 void decode_geometry(int B, int Hkv, int max_blocks, int* tiles_per_split, int* num_splits) {
   // Aim at about two resident CTAs per SM on a 148-SM part, four tiles per CTA at least.

@@ -178,6 +178,26 @@ kvarn_status kvarn_decode_attention(const void* q, const void* packed_cache, con
   return from_cuda(kvarn::launch_decode(p, static_cast<cudaStream_t>(stream)));
 }
 
+kvarn_status kvarn_decode_attention_noalloc(const void* q, const void* packed_cache, const void* scales,
+                                            const void* fp16_tail, const int32_t* block_table,
+                                            const int32_t* seq_lens, void* out, const kvarn_decode_dims* dims,
+                                            const kvarn_config* cfg, int32_t* dev_status, void* stream) {
+  // Same path as kvarn_decode_attention, with the library's fixed device
+  // scratch standing in for the caller's workspace.
+  kvarn_status st = kvarn_config_validate(cfg);
+  if (st != KVARN_OK) return st;
+  st = check_dims(dims, 8);
+  if (st != KVARN_OK) return st;
+  if (dims->num_seqs == 0) return KVARN_OK;
+  const size_t need = workspace_for(dims->num_seqs, dims->num_q_heads, dims->num_kv_heads, dims->max_blocks_per_seq);
+  if (need > kvarn::kNoAllocScratchBytes) return KVARN_ERR_WORKSPACE_TOO_SMALL;
+  void* scratch = nullptr;
+  size_t scratch_bytes = 0;
+  if (kvarn::noalloc_scratch(&scratch, &scratch_bytes) != cudaSuccess) return KVARN_ERR_CUDA;
+  return kvarn_decode_attention(q, packed_cache, scales, fp16_tail, block_table, seq_lens, out, dims, cfg, scratch,
+                                scratch_bytes, dev_status, stream);
+}
+
 size_t kvarn_baseline_workspace_bytes(const kvarn_decode_dims* dims) {
   if (check_dims(dims, 8) != KVARN_OK) return 0;
   return workspace_for(dims->num_seqs, dims->num_q_heads, dims->num_kv_heads, dims->max_blocks_per_seq);

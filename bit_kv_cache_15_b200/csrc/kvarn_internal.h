@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "../../include/kvarn.h"
+
 namespace kvarn {
 
 struct QuantArgs {
@@ -46,6 +48,12 @@ struct DecodeArgs {
 void decode_geometry(int B, int Hkv, int max_blocks, int* tiles_per_split, int* num_splits);
 
 cudaError_t launch_quantize(const QuantArgs& p, cudaStream_t stream);
+
+// Fixed device scratch of kvarn_decode_attention_noalloc (KVARN_NOALLOC_SCRATCH_BYTES).
+constexpr size_t kNoAllocScratchBytes = KVARN_NOALLOC_SCRATCH_BYTES;
+// Device address and size of that scratch on the current device; the first
+// call on a device looks the address up (cudaGetSymbolAddress) and caches it.
+cudaError_t noalloc_scratch(void** ptr, size_t* bytes);
 cudaError_t launch_decode(const DecodeArgs& p, cudaStream_t stream);
 
 struct BaselineArgs {

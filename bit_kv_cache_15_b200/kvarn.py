@@ -61,6 +61,8 @@ _SIGS = {
                                          _vp, _vp, _vp]),
     "kvarn_decode_attention": (_st, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(DecodeDims),
                                      ctypes.POINTER(Config), _vp, _sz, _vp, _vp]),
+    "kvarn_decode_attention_noalloc": (_st, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(DecodeDims),
+                                             ctypes.POINTER(Config), _vp, _vp]),
     "kvarn_baseline_workspace_bytes": (_sz, [ctypes.POINTER(DecodeDims)]),
     "kvarn_decode_attention_fp16": (_st, [_vp, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(DecodeDims),
                                           ctypes.c_float, _vp, _sz, _vp, _vp]),
@@ -195,6 +197,29 @@ def decode_attention(q: torch.Tensor, packed_cache: torch.Tensor, scales: torch.
                                      _ptr(workspace), workspace.numel() * workspace.element_size(),
                                      _ptr(dev_status), _stream(stream))
     _check("kvarn_decode_attention", st)
+    return out
+
+
+def decode_attention_noalloc(q: torch.Tensor, packed_cache: torch.Tensor, scales: torch.Tensor,
+                             fp16_tail: torch.Tensor, block_table: torch.Tensor, seq_lens: torch.Tensor, cfg: Config,
+                             out: torch.Tensor | None = None, dev_status: torch.Tensor | None = None,
+                             stream=None) -> torch.Tensor:
+    """decode_attention with the library's fixed device scratch instead of a
+    workspace tensor (see kvarn_decode_attention_noalloc in include/kvarn.h)."""
+    _need(q, "q", torch.float16)
+    _need(packed_cache, "packed_cache", torch.uint8)
+    _need(scales, "scales", torch.uint8)
+    _need(fp16_tail, "fp16_tail", torch.float16)
+    _need(block_table, "block_table", torch.int32)
+    _need(seq_lens, "seq_lens", torch.int32)
+    B, Hq, _ = q.shape
+    d = dims(B, Hq, int(packed_cache.shape[1]), int(block_table.shape[1]), int(packed_cache.shape[0]))
+    if out is None:
+        out = torch.empty_like(q)
+    st = _lib.kvarn_decode_attention_noalloc(_ptr(q), _ptr(packed_cache), _ptr(scales), _ptr(fp16_tail),
+                                             _ptr(block_table), _ptr(seq_lens), _ptr(out), ctypes.byref(d),
+                                             ctypes.byref(cfg), _ptr(dev_status), _stream(stream))
+    _check("kvarn_decode_attention_noalloc", st)
     return out
 
 

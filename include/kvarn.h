@@ -162,6 +162,36 @@ KVARN_API kvarn_status kvarn_decode_attention(const void* q, const void* packed_
                                     void* workspace, size_t workspace_bytes,
                                     int32_t* dev_status, void* stream);
 
+/* Size of the fixed device scratch used by kvarn_decode_attention_noalloc. */
+#define KVARN_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+/* kvarn_decode_attention without a workspace argument: the call allocates
+ * nothing.  (The pages have no counterpart; this is a convenience of this
+ * library.)  It is meant for callers that cannot allocate device memory
+ * themselves -- for instance code running inside another framework's step
+ * that owns all allocations, or a host thread that must not call cudaMalloc
+ * because that can synchronise the device.  The split-K scratch is instead a
+ * file-scope __device__ array of KVARN_NOALLOC_SCRATCH_BYTES (8 MiB) that
+ * every GPU loading this library keeps until the process exits.
+ *  - Same arguments and results as kvarn_decode_attention, minus workspace.
+ *  - If the problem needs more scratch than that (kvarn_decode_workspace_bytes
+ *    > KVARN_NOALLOC_SCRATCH_BYTES) the call returns
+ *    KVARN_ERR_WORKSPACE_TOO_SMALL and launches nothing.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current and caches it; make that
+ *    first call before any stream capture begins.
+ *  - All calls on a device share the one array and it keeps the previous
+ *    call's contents.  Nothing in it needs to start at zero: every record a
+ *    call reads was written earlier in the same call.  Calls whose kernels
+ *    overlap on the GPU (different streams, no ordering) race on the array;
+ *    order them on one stream or by events.
+ *  - It calls no cudaMalloc, cudaFree or other allocating routine. */
+KVARN_API kvarn_status kvarn_decode_attention_noalloc(const void* q, const void* packed_cache, const void* scales,
+                                                      const void* fp16_tail, const int32_t* block_table,
+                                                      const int32_t* seq_lens, void* out,
+                                                      const kvarn_decode_dims* dims, const kvarn_config* cfg,
+                                                      int32_t* dev_status, void* stream);
+
 /* Measurement baselines: the same paged decode over UNCOMPRESSED caches.
  *  k_cache, v_cache  [num_blocks][Hkv][128 tokens][128] fp16 (or fp8 e4m3 for
  *                    the _fp8 variant, values = e4m3 * k_scale / v_scale);
