@@ -286,7 +286,7 @@ def run_gpu(args):
                        "l2": f"inputs larger than L2: {(q_bytes + d_bytes) / 1e6:.0f} MB of algorithmic traffic per step"},
             "e2e": {"value": world * BATCH * args.steps / (ms_e2e * 1e-3), "unit": "decode tokens/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": 3 * args.steps,
+            "gpu_launches": 3 * args.steps,   # quantize kernel, counter memset, decode kernel
             "roofline": {"bound": "hbm", "kernel": dominant, "achieved": dom_gbs, "peak": hbm_peak,
                          "unit": "GB/s", "frac": dom_gbs / hbm_peak, "traffic": traffic,
                          "peak_kind": f"{peak_kind} (burst copy)"},

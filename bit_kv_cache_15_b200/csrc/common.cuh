@@ -68,6 +68,13 @@ __device__ __forceinline__ uint32_t pack_f2h2(float lo, float hi) {
   return h2_as_u32(__floats2half2_rn(lo, hi));
 }
 
+// 2^x on the SFU (MUFU.EX2): about 2 ulp, flushes subnormal results, 2^-inf = 0.
+__device__ __forceinline__ float ex2_fast(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));

@@ -126,7 +126,7 @@ __device__ void decode_tail(const DecodeArgs& p, uint8_t* smem, float* qs, int b
     float l = 0.f;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const float e = exp2f(v[i] - m);
+      const float e = ex2_fast(v[i] - m);
       sc[g * 128 + lane + 32 * i] = e;
       l += e;
     }
@@ -161,27 +161,18 @@ __device__ void decode_tail(const DecodeArgs& p, uint8_t* smem, float* qs, int b
 
 // ------------------------------------------------------------------ main kernel
 
+// One split: tiles [s*T, s*T + T) of sequence b, KV head h; writes one
+// partial record per query head (or nothing if the split is empty).
 template <int KB, int VB>
-__global__ void __launch_bounds__(kDThreads, 2) decode_kernel(const DecodeArgs p) {
+__device__ __forceinline__ void decode_split(const DecodeArgs& p, uint8_t* smem, int b, int h, int s, int L) {
   using T = DecodeTraits<KB, VB>;
   constexpr int U = T::U, MT = T::MT;
-  extern __shared__ __align__(128) uint8_t smem[];
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + T::kBarOff);
   float* qrot = reinterpret_cast<float*>(smem + T::kQrotOff);
   float* invsig = reinterpret_cast<float*>(smem + T::kInvSigOff);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int G = p.G;
-  const int L = p.seq_lens[b];
-  if (L < 0 || L > kTile * p.max_blocks) {
-    if (tid == 0 && s == 0) report_status(p.status, KVARN_DEV_BAD_SEQ_LEN);
-    return;
-  }
-  if (s == p.num_splits) {
-    decode_tail(p, smem, qrot, b, h, L);
-    return;
-  }
   const int n_full = L >> 7;
   const int t_begin = s * p.tiles_per_split;
   const int t_end = min(t_begin + p.tiles_per_split, n_full);
@@ -301,7 +292,7 @@ __global__ void __launch_bounds__(kDThreads, 2) decode_kernel(const DecodeArgs p
 
   for (int k = 0; k < n_mine; ++k) {
     const int stg = k & 1;
-    if (!mbar_wait_bounded(&my_bars[stg], (k >> 1) & 1)) {
+    if (!__all_sync(0xffffffffu, mbar_wait_bounded(&my_bars[stg], (k >> 1) & 1))) {
       if (lane == 0) report_status(p.status, KVARN_DEV_TIMEOUT);
       k_fail = k;
       break;
@@ -330,7 +321,7 @@ __global__ void __launch_bounds__(kDThreads, 2) decode_kernel(const DecodeArgs p
       }
       const float E = ceilf(warp_max(fmaxf(fmaxf(lcl[0], lcl[1]), fmaxf(lcl[2], lcl[3]))));
       *reinterpret_cast<float4*>(&scr[4 * lane]) =
-          make_float4(exp2f(lcl[0] - E), exp2f(lcl[1] - E), exp2f(lcl[2] - E), exp2f(lcl[3] - E));
+          make_float4(ex2_fast(lcl[0] - E), ex2_fast(lcl[1] - E), ex2_fast(lcl[2] - E), ex2_fast(lcl[3] - E));
       __syncwarp();
       // q' as an fp16 hi + lo pair (about 22 significant bits): scores can reach
       // |s| ~ 10 nats, where plain fp16 q' would cost ~1e-2 in the output
@@ -401,8 +392,8 @@ __global__ void __launch_bounds__(kDThreads, 2) decode_kernel(const DecodeArgs p
 #pragma unroll
         for (int ri = 0; ri < 2; ++ri) {
           const int t = t0 + 16 * mt + g8 + 8 * ri;
-          const float tk = exp2f(hf(ltk, t));
-          tv[mt][ri] = exp2f(hf(ltv, t));
+          const float tk = ex2_fast(hf(ltk, t));
+          tv[mt][ri] = ex2_fast(hf(ltv, t));
           S[mt][2 * ri] = fmaf(sk, S[mt][2 * ri], za0) * (cf0 * tk);
           S[mt][2 * ri + 1] = fmaf(sk, S[mt][2 * ri + 1], za1) * (cf1 * tk);
           mx0 = fmaxf(mx0, S[mt][2 * ri]);
@@ -414,7 +405,7 @@ __global__ void __launch_bounds__(kDThreads, 2) decode_kernel(const DecodeArgs p
         mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
       }
       const float mn0 = fmaxf(mrun[0], mx0), mn1 = fmaxf(mrun[1], mx1);
-      const float al0 = exp2f(mrun[0] - mn0), al1 = exp2f(mrun[1] - mn1);
+      const float al0 = ex2_fast(mrun[0] - mn0), al1 = ex2_fast(mrun[1] - mn1);
       mrun[0] = mn0;
       mrun[1] = mn1;
       float ls0 = 0.f, ls1 = 0.f, ps0 = 0.f, ps1 = 0.f;
@@ -424,8 +415,8 @@ __global__ void __launch_bounds__(kDThreads, 2) decode_kernel(const DecodeArgs p
         uint32_t pk[2];
 #pragma unroll
         for (int ri = 0; ri < 2; ++ri) {
-          const float p0 = exp2f(S[mt][2 * ri] - mn0);
-          const float p1 = exp2f(S[mt][2 * ri + 1] - mn1);
+          const float p0 = ex2_fast(S[mt][2 * ri] - mn0);
+          const float p1 = ex2_fast(S[mt][2 * ri + 1] - mn1);
           ls0 += p0;
           ls1 += p1;
           const __half2 hp = __floats2half2_rn(p0 * tv[mt][ri], p1 * tv[mt][ri]);
@@ -481,7 +472,7 @@ __global__ void __launch_bounds__(kDThreads, 2) decode_kernel(const DecodeArgs p
       for (int mt = 0; mt < 8; ++mt)
 #pragma unroll
         for (int ri = 0; ri < 2; ++ri) {
-          const float vcs = exp2f(hf(lcv, 16 * mt + g8 + 8 * ri));
+          const float vcs = ex2_fast(hf(lcv, 16 * mt + g8 + 8 * ri));
           acc[mt][2 * ri] = fmaf(acc[mt][2 * ri], al0, vcs * fmaf(sv, O[mt][2 * ri], zp0));
           acc[mt][2 * ri + 1] = fmaf(acc[mt][2 * ri + 1], al1, vcs * fmaf(sv, O[mt][2 * ri + 1], zp1));
         }
@@ -533,7 +524,7 @@ __global__ void __launch_bounds__(kDThreads, 2) decode_kernel(const DecodeArgs p
 #pragma unroll
     for (int w = 0; w < kDWarps; ++w) {
       const float mw = mS[w * kMaxG + g];
-      const float f = mw == -INFINITY ? 0.f : exp2f(mw - M);
+      const float f = mw == -INFINITY ? 0.f : ex2_fast(mw - M);
       l = fmaf(f, lS[w * kMaxG + g], l);
       a = fmaf(f, aS[(w * kMaxG + g) * kHeadDim + d], a);
     }
@@ -550,64 +541,95 @@ __global__ void __launch_bounds__(kDThreads, 2) decode_kernel(const DecodeArgs p
 
 // ------------------------------------------------------------------ combine (a10)
 
-__global__ void __launch_bounds__(128) combine_kernel(const DecodeArgs p) {
-  const int wg = blockIdx.x * 4 + (threadIdx.x >> 5);
-  if (wg >= p.B * p.Hq) return;
-  const int lane = threadIdx.x & 31;
-  const int b = wg / p.Hq, j = wg % p.Hq;
-  int L = p.seq_lens[b];
-  __half* o = p.out + ((int64_t)b * p.Hq + j) * kHeadDim + 4 * lane;
-  if (L <= 0 || L > kTile * p.max_blocks) {
-    *reinterpret_cast<uint2*>(o) = make_uint2(0u, 0u);
-    return;
-  }
-  const int n_full = L >> 7;
-  const int nsv = (n_full + p.tiles_per_split - 1) / p.tiles_per_split;
-  const bool has_tail = (L & 127) != 0;
-  const float* rec = p.ws + ((int64_t)b * p.Hq + j) * (p.num_splits + 1) * kPartialFloats;
-  const float* trec = rec + (int64_t)p.num_splits * kPartialFloats;
-  float M = has_tail ? trec[0] : -INFINITY;
-  for (int s = 0; s < nsv; ++s) M = fmaxf(M, rec[(int64_t)s * kPartialFloats]);
-  float l = 0.f, a[4] = {0.f, 0.f, 0.f, 0.f};
-  for (int s = 0; s < nsv; ++s) {
-    const float* r = rec + (int64_t)s * kPartialFloats;
-    const float w = exp2f(r[0] - M);
-    l = fmaf(w, r[1], l);
-    const float4 v = *reinterpret_cast<const float4*>(r + 4 + 4 * lane);
-    a[0] = fmaf(w, v.x, a[0]);
-    a[1] = fmaf(w, v.y, a[1]);
-    a[2] = fmaf(w, v.z, a[2]);
-    a[3] = fmaf(w, v.w, a[3]);
-  }
-  // acc H / 128: channels 4*lane .. 4*lane+3 in this lane
-  {
-    float b0 = a[0] + a[1], b1 = a[0] - a[1], b2 = a[2] + a[3], b3 = a[2] - a[3];
-    a[0] = b0 + b2; a[1] = b1 + b3; a[2] = b0 - b2; a[3] = b1 - b3;
-#pragma unroll
-    for (int m = 1; m < 32; m <<= 1) {
-      const bool up = (lane & m) != 0;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float y = __shfl_xor_sync(0xffffffffu, a[i], m);
-        a[i] = up ? (y - a[i]) : (a[i] + y);
-      }
+// Merge the partials of (b, h) for its G query heads: o = (acc H / 128 + tail) / l.
+// One warp per head; lane owns channels 4*lane .. 4*lane + 3.  Records written
+// by other CTAs are read with ld.global.cg (L2), never through L1.
+__device__ void combine_pair(const DecodeArgs& p, int b, int h, int L, bool valid) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int g = warp; g < p.G; g += kDWarps) {
+    const int j = h * p.G + g;
+    __half* o = p.out + ((int64_t)b * p.Hq + j) * kHeadDim + 4 * lane;
+    if (!valid || L == 0) {
+      *reinterpret_cast<uint2*>(o) = make_uint2(0u, 0u);
+      continue;
     }
+    const int n_full = L >> 7;
+    const int nsv = (n_full + p.tiles_per_split - 1) / p.tiles_per_split;
+    const bool has_tail = (L & 127) != 0;
+    const float* rec = p.ws + ((int64_t)b * p.Hq + j) * (p.num_splits + 1) * kPartialFloats;
+    const float* trec = rec + (int64_t)p.num_splits * kPartialFloats;
+    float M = has_tail ? __ldcg(trec) : -INFINITY;
+    for (int s = 0; s < nsv; ++s) M = fmaxf(M, __ldcg(rec + (int64_t)s * kPartialFloats));
+    float l = 0.f, a[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int s = 0; s < nsv; ++s) {
+      const float* r = rec + (int64_t)s * kPartialFloats;
+      const float w = ex2_fast(__ldcg(r) - M);
+      l = fmaf(w, __ldcg(r + 1), l);
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(r + 4 + 4 * lane));
+      a[0] = fmaf(w, v.x, a[0]);
+      a[1] = fmaf(w, v.y, a[1]);
+      a[2] = fmaf(w, v.z, a[2]);
+      a[3] = fmaf(w, v.w, a[3]);
+    }
+    {   // acc H / 128
+      const float b0 = a[0] + a[1], b1 = a[0] - a[1], b2 = a[2] + a[3], b3 = a[2] - a[3];
+      a[0] = b0 + b2; a[1] = b1 + b3; a[2] = b0 - b2; a[3] = b1 - b3;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) a[i] *= (1.f / 128.f);
+      for (int m = 1; m < 32; m <<= 1) {
+        const bool up = (lane & m) != 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float y = __shfl_xor_sync(0xffffffffu, a[i], m);
+          a[i] = up ? (y - a[i]) : (a[i] + y);
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[i] *= (1.f / 128.f);
+    }
+    if (has_tail) {
+      const float w = ex2_fast(__ldcg(trec) - M);
+      l = fmaf(w, __ldcg(trec + 1), l);
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(trec + 4 + 4 * lane));
+      a[0] = fmaf(w, v.x, a[0]);
+      a[1] = fmaf(w, v.y, a[1]);
+      a[2] = fmaf(w, v.z, a[2]);
+      a[3] = fmaf(w, v.w, a[3]);
+    }
+    const float il = 1.f / l;
+    const __half2 o01 = __floats2half2_rn(a[0] * il, a[1] * il);
+    const __half2 o23 = __floats2half2_rn(a[2] * il, a[3] * il);
+    *reinterpret_cast<uint2*>(o) = make_uint2(h2_as_u32(o01), h2_as_u32(o23));
   }
-  if (has_tail) {
-    const float w = exp2f(trec[0] - M);
-    l = fmaf(w, trec[1], l);
-    const float4 v = *reinterpret_cast<const float4*>(trec + 4 + 4 * lane);
-    a[0] = fmaf(w, v.x, a[0]);
-    a[1] = fmaf(w, v.y, a[1]);
-    a[2] = fmaf(w, v.z, a[2]);
-    a[3] = fmaf(w, v.w, a[3]);
+}
+
+// Grid (num_splits + 1, Hkv, B).  Every CTA of (b, h) -- empty splits and the
+// tail CTA included -- bumps the pair's counter (cleared before the launch)
+// once after its records are visible; the last of the num_splits + 1 arrivals
+// merges them.  Nothing waits on anything.
+template <int KB, int VB>
+__global__ void __launch_bounds__(kDThreads, 2) decode_kernel(const DecodeArgs p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ int last_arrival;
+  const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int L = p.seq_lens[b];
+  const bool valid = L >= 0 && L <= kTile * p.max_blocks;
+  if (!valid) {
+    if (threadIdx.x == 0 && s == 0) report_status(p.status, KVARN_DEV_BAD_SEQ_LEN);
+  } else if (s == p.num_splits) {
+    decode_tail(p, smem, reinterpret_cast<float*>(smem + DecodeTraits<KB, VB>::kQrotOff), b, h, L);
+  } else {
+    decode_split<KB, VB>(p, smem, b, h, s, L);
   }
-  const float il = 1.f / l;
-  const __half2 o01 = __floats2half2_rn(a[0] * il, a[1] * il);
-  const __half2 o23 = __floats2half2_rn(a[2] * il, a[3] * il);
-  *reinterpret_cast<uint2*>(o) = make_uint2(h2_as_u32(o01), h2_as_u32(o23));
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int* cnt = p.counters + (int64_t)b * p.Hkv + h;
+    last_arrival = atomicAdd(cnt, 1) == p.num_splits;
+  }
+  __syncthreads();
+  if (!last_arrival) return;
+  __threadfence();
+  combine_pair(p, b, h, L, valid);
 }
 
 template <int KB, int VB>
@@ -623,12 +645,11 @@ cudaError_t launch_d(const DecodeArgs& p, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     configured.fetch_or(bit, std::memory_order_acq_rel);
   }
+  // the per-(seq, KV head) arrival counters start every call at zero
+  cudaError_t e = cudaMemsetAsync(p.counters, 0, static_cast<size_t>(p.B) * p.Hkv * sizeof(int), stream);
+  if (e != cudaSuccess) return e;
   const dim3 grid(static_cast<unsigned>(p.num_splits + 1), static_cast<unsigned>(p.Hkv), static_cast<unsigned>(p.B));
   decode_kernel<KB, VB><<<grid, kDThreads, T::kSmem, stream>>>(p);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  const unsigned nc = static_cast<unsigned>((p.B * p.Hq + 3) / 4);
-  combine_kernel<<<nc, 128, 0, stream>>>(p);
   return cudaGetLastError();
 }
 
@@ -661,15 +682,26 @@ cudaError_t noalloc_scratch(void** ptr, size_t* bytes) {
 }
 
 void decode_geometry(int B, int Hkv, int max_blocks, int* tiles_per_split, int* num_splits) {
-  // Aim at about two resident CTAs per SM on a 148-SM part, four tiles per CTA at least.
-  const int pairs = B * Hkv > 0 ? B * Hkv : 1;
-  const int target = 2 * 148 * 2;
-  const int want = (target + pairs - 1) / pairs;
-  int T = (max_blocks + want - 1) / want;
-  if (T < kDWarps) T = kDWarps;
-  int ns = (max_blocks + T - 1) / T;
+  // Tiles per split T (a multiple of the 4 warps) chosen to minimise
+  // waves x (T / 4 tiles per warp + one tile of fixed cost), with about two
+  // resident CTAs per SM on a 148-SM part; ties go to the larger T.
+  const long pairs = B * Hkv > 0 ? static_cast<long>(B) * Hkv : 1;
+  const long slots = 2 * 148;
+  int best_t = kDWarps;
+  double best = 1e300;
+  for (int T = kDWarps; T <= 64; T += kDWarps) {
+    const long ns = (max_blocks + T - 1) / T;
+    const long waves = (pairs * ns + slots - 1) / slots;
+    const double cost = static_cast<double>(waves) * (T / static_cast<double>(kDWarps) + 1.0);
+    if (cost <= best) {
+      best = cost;
+      best_t = T;
+    }
+    if (ns == 1) break;
+  }
+  int ns = (max_blocks + best_t - 1) / best_t;
   if (ns < 1) ns = 1;
-  *tiles_per_split = T;
+  *tiles_per_split = best_t;
   *num_splits = ns;
 }
 

@@ -37,10 +37,16 @@ kvarn_status check_dims(const kvarn_decode_dims* dims, int max_group) {
 
 kvarn_status from_cuda(cudaError_t e) { return e == cudaSuccess ? KVARN_OK : KVARN_ERR_CUDA; }
 
-size_t workspace_for(int B, int Hq, int Hkv, int max_blocks) {
+size_t partial_bytes(int B, int Hq, int Hkv, int max_blocks) {
   int T = 0, ns = 0;
   kvarn::decode_geometry(B, Hkv, max_blocks, &T, &ns);
   return static_cast<size_t>(B) * Hq * (ns + 1) * kvarn::kPartialFloats * sizeof(float);
+}
+
+// partial records followed by B * Hkv int32 arrival counters (rounded to 16 bytes)
+size_t workspace_for(int B, int Hq, int Hkv, int max_blocks) {
+  const size_t counters = (static_cast<size_t>(B) * Hkv * sizeof(int32_t) + 15) & ~static_cast<size_t>(15);
+  return partial_bytes(B, Hq, Hkv, max_blocks) + counters;
 }
 
 kvarn_status quantize_impl(const void* k, const void* v, const int64_t* slot_mapping, int64_t num_tokens,
@@ -164,6 +170,9 @@ kvarn_status kvarn_decode_attention(const void* q, const void* packed_cache, con
   p.seq_lens = seq_lens;
   p.out = static_cast<__half*>(out);
   p.ws = static_cast<float*>(workspace);
+  p.counters = reinterpret_cast<int*>(static_cast<uint8_t*>(workspace) +
+                                      partial_bytes(dims->num_seqs, dims->num_q_heads, dims->num_kv_heads,
+                                                    dims->max_blocks_per_seq));
   p.B = dims->num_seqs;
   p.Hq = dims->num_q_heads;
   p.Hkv = dims->num_kv_heads;

@@ -35,7 +35,8 @@ struct DecodeArgs {
   const int32_t* block_table;
   const int32_t* seq_lens;
   __half* out;
-  float* ws;
+  float* ws;            // partial records, then the per-(seq, KV head) counters
+  int* counters;        // B * Hkv arrival counters (zero between calls)
   int B, Hq, Hkv, G, max_blocks;
   int64_t num_blocks;
   int kb, vb;

@@ -1,18 +1,19 @@
 // quantize.cu -- KVarN quantise-on-write for whole 128-token tiles (sm_100a).
 //
-// One CTA (4 warps) per (token group, KV head, K|V) tile.  The four stages of
-// [hypho] "KV-cache 量化终于能跑生产了？KVarN …" section 它怎么做到的：四步流水线
-// (= [lehuy] "KVarN: Backend lượng tử hóa KV-cache …" section Cơ chế hoạt động):
-//   1 stage   the fp16 tile in shared memory (16-byte chunks XOR-swizzled by
-//             row so ldmatrix is conflict-free);
+// The four stages of [hypho] "KV-cache 量化终于能跑生产了？KVarN …", section
+// 它怎么做到的：四步流水线 (= [lehuy] "KVarN: Backend lượng tử hóa KV-cache …",
+// section Cơ chế hoạt động), one (token group, KV head, K|V) tile at a time:
+//   1 stage   the fp16 tile is brought into shared memory by the TMA engine
+//             (cp.async.bulk.tensor, two 64-channel boxes, 128-byte swizzle so
+//             ldmatrix reads are conflict-free).  CTAs are persistent and load
+//             the next tile while they compute the current one;
 //   2 rotate  R = X H along channels.  H128 = H8 (x) H16 (Kronecker), so the
 //             16-channel factor runs on the tensor cores (mma.m16n8k16 against
 //             a +-1 fp16 H16) and the 8-group factor is an in-register
 //             butterfly across the eight mma results each lane holds;
 //   3 normalise  N passes of channel RMS then token RMS in base-2 log space:
-//             A = R*R stays in registers; per pass every lane does its FMAs,
-//             then a warp reduce-scatter (and, for channels, a 4-warp shared
-//             memory sum) yields one scale per lane or per thread;
+//             A = R*R stays in registers; each pass is packed f32x2 FMAs, a
+//             warp reduce-scatter and (for channels) a 4-warp shared sum;
 //   4 quantise   Z = (R * fp32(2^-Lt)) * fp32(2^-Lc) from the stored fp16
 //             log-scales, one zero/step per tile from min/max, codes =
 //             clamp(rne((Z - zero) * (1/step))).
@@ -20,6 +21,12 @@
 // operand, so after stage 2 each lane holds exactly the elements of the
 // decode kernel's mma fragments (K: rows tokens; V: rows channels): codes are
 // packed in registers and written with 16-byte stores, no cross-lane traffic.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <mutex>
+
 #include "common.cuh"
 #include "kvarn_internal.h"
 
@@ -27,16 +34,34 @@ namespace kvarn {
 namespace {
 
 constexpr int kQThreads = 128;
+constexpr int kBox = 128 * 128;       // one 64-channel box: 128 rows of 128 bytes
 
 struct QuantSmem {
-  alignas(128) uint8_t x[kTile * 256];  // fp16 tile, row t at t*256, chunk c at (c ^ (t&7))*16
+  alignas(1024) uint8_t x[2][2][kBox];  // [stage][channel half] swizzled fp16 tile
   float red[4][kHeadDim];                // per-warp channel partial sums
   float u[kHeadDim];                     // channel weights 2^(-2 lc)
   float mt[kTile];                       // fp32(2^-Lt)
   float mc[kHeadDim];                    // fp32(2^-Lc)
   float zmin[4], zmax[4];
   alignas(16) uint8_t rec[kScaleRec];    // staged scale record
+  alignas(8) uint64_t bar[2];
 };
+
+// byte offset of (row t, 16-byte chunk c16 in 0..15) inside one stage
+__device__ __forceinline__ uint32_t xoff(int t, int c16) {
+  return (c16 >> 3) * kBox + t * 128 + (((c16 & 7) ^ (t & 7)) << 4);
+}
+
+__device__ __forceinline__ float lg2_approx(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// 1/2 log2 of the mean square (sum / 128), floored at 2^-48
+__device__ __forceinline__ float log2_scale(float sum_sq) {
+  return 0.5f * (lg2_approx(fmaxf(sum_sq, 4.547473508864641e-13f)) - 7.0f);   // 2^-41
+}
 
 // fp16 bit pattern of the Hadamard sign H16[r][c] = (-1)^popcount(r & c).
 __device__ __forceinline__ uint32_t h16_bits(int r, int c) {
@@ -46,16 +71,17 @@ __device__ __forceinline__ uint32_t h16_pair(int r0, int c0, int r1, int c1) {
   return h16_bits(r0, c0) | (h16_bits(r1, c1) << 16);
 }
 
-// In-register 8-point Walsh-Hadamard transform (Sylvester order).
-__device__ __forceinline__ void fwht8(float (&v)[8]) {
+// In-register 8-point Walsh-Hadamard transforms (Sylvester order) of two
+// independent vectors at once: lane .x of v is one vector, lane .y the other.
+__device__ __forceinline__ void fwht8x2(float2 (&v)[8]) {
 #pragma unroll
   for (int hl = 1; hl < 8; hl <<= 1) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       if ((i & hl) == 0) {
-        const float a = v[i], b = v[i + hl];
-        v[i] = a + b;
-        v[i + hl] = a - b;
+        const float2 a = v[i], b = v[i + hl];
+        v[i] = __fadd2_rn(a, b);
+        v[i + hl] = __fadd2_rn(a, make_float2(-b.x, -b.y));
       }
     }
   }
@@ -74,16 +100,20 @@ __device__ __forceinline__ void rs_step(float* v, int mask, int lane) {
   }
 }
 
-__device__ __forceinline__ float log2_scale(float sum_sq) {
-  // half log2 of the mean square, floored at 2^-48
-  return 0.5f * __log2f(fmaxf(sum_sq * (1.0f / 128.0f), 3.552713678800501e-15f));
+__device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
+
+// insert the low `len` bits of x into y at bit `pos`
+__device__ __forceinline__ uint32_t bfi(uint32_t x, uint32_t y, int pos, int len) {
+  uint32_t r;
+  asm("bfi.b32 %0, %1, %2, %3, %4;\n" : "=r"(r) : "r"(x), "r"(y), "r"(pos), "r"(len));
+  return r;
 }
 
 // ---------------------------------------------------------------- rotation
 
 // K side: thread holds R at t = 16*(2w+ml) + g + 8*ri, d = 16*a + 8*nb + 2*c + rj
 // in R[((ml*8 + a)*2 + nb)*4 + 2*ri + rj]   (g = lane/4, c = lane%4).
-__device__ __forceinline__ void rotate_k(const QuantSmem& sm, int warp, int lane, float (&R)[128]) {
+__device__ __forceinline__ void rotate_k(uint32_t xs, int warp, int lane, float (&R)[128]) {
   const int g = lane >> 2, c = lane & 3;
   uint32_t hb0[2], hb1[2];
 #pragma unroll
@@ -92,7 +122,6 @@ __device__ __forceinline__ void rotate_k(const QuantSmem& sm, int warp, int lane
     hb0[nb] = h16_pair(2 * c, n, 2 * c + 1, n);
     hb1[nb] = h16_pair(2 * c + 8, n, 2 * c + 9, n);
   }
-  const uint32_t xbase = smem_u32(sm.x);
   const int mi = lane >> 3;
 #pragma unroll
   for (int ml = 0; ml < 2; ++ml) {
@@ -100,9 +129,8 @@ __device__ __forceinline__ void rotate_k(const QuantSmem& sm, int warp, int lane
     float C[8][2][4];
 #pragma unroll
     for (int a = 0; a < 8; ++a) {
-      const int chunk = 2 * a + (mi >> 1);
       uint32_t a0, a1, a2, a3;
-      ldmatrix_x4(xbase + row * 256 + ((chunk ^ (row & 7)) << 4), a0, a1, a2, a3);
+      ldmatrix_x4(xs + xoff(row, 2 * a + (mi >> 1)), a0, a1, a2, a3);
 #pragma unroll
       for (int nb = 0; nb < 2; ++nb) {
 #pragma unroll
@@ -113,13 +141,16 @@ __device__ __forceinline__ void rotate_k(const QuantSmem& sm, int warp, int lane
 #pragma unroll
     for (int nb = 0; nb < 2; ++nb) {
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        float v[8];
+      for (int r = 0; r < 4; r += 2) {
+        float2 v[8];
 #pragma unroll
-        for (int a = 0; a < 8; ++a) v[a] = C[a][nb][r];
-        fwht8(v);
+        for (int a = 0; a < 8; ++a) v[a] = make_float2(C[a][nb][r], C[a][nb][r + 1]);
+        fwht8x2(v);
 #pragma unroll
-        for (int a = 0; a < 8; ++a) R[((ml * 8 + a) * 2 + nb) * 4 + r] = v[a];
+        for (int a = 0; a < 8; ++a) {
+          R[((ml * 8 + a) * 2 + nb) * 4 + r] = v[a].x;
+          R[((ml * 8 + a) * 2 + nb) * 4 + r + 1] = v[a].y;
+        }
       }
     }
   }
@@ -127,13 +158,12 @@ __device__ __forceinline__ void rotate_k(const QuantSmem& sm, int warp, int lane
 
 // V side: thread holds R at t = 8*(4w+ntl) + 2*c + rj, d = 16*a + g + 8*ri
 // in R[(ntl*8 + a)*4 + 2*ri + rj].
-__device__ __forceinline__ void rotate_v(const QuantSmem& sm, int warp, int lane, float (&R)[128]) {
+__device__ __forceinline__ void rotate_v(uint32_t xs, int warp, int lane, float (&R)[128]) {
   const int g = lane >> 2, c = lane & 3;
   const uint32_t ha0 = h16_pair(g, 2 * c, g, 2 * c + 1);
   const uint32_t ha1 = h16_pair(g + 8, 2 * c, g + 8, 2 * c + 1);
   const uint32_t ha2 = h16_pair(g, 2 * c + 8, g, 2 * c + 9);
   const uint32_t ha3 = h16_pair(g + 8, 2 * c + 8, g + 8, 2 * c + 9);
-  const uint32_t xbase = smem_u32(sm.x);
   const int mi = lane >> 3;
 #pragma unroll
   for (int ntl = 0; ntl < 4; ++ntl) {
@@ -141,9 +171,8 @@ __device__ __forceinline__ void rotate_v(const QuantSmem& sm, int warp, int lane
     float C[8][4];
 #pragma unroll
     for (int ap = 0; ap < 4; ++ap) {
-      const int chunk = 4 * ap + mi;
       uint32_t r0, r1, r2, r3;
-      ldmatrix_x4(xbase + row * 256 + ((chunk ^ (row & 7)) << 4), r0, r1, r2, r3);
+      ldmatrix_x4(xs + xoff(row, 4 * ap + mi), r0, r1, r2, r3);
 #pragma unroll
       for (int r = 0; r < 4; ++r) {
         C[2 * ap][r] = 0.f;
@@ -153,13 +182,16 @@ __device__ __forceinline__ void rotate_v(const QuantSmem& sm, int warp, int lane
       mma_f16(C[2 * ap + 1], ha0, ha1, ha2, ha3, r2, r3);
     }
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      float v[8];
+    for (int r = 0; r < 4; r += 2) {
+      float2 v[8];
 #pragma unroll
-      for (int a = 0; a < 8; ++a) v[a] = C[a][r];
-      fwht8(v);
+      for (int a = 0; a < 8; ++a) v[a] = make_float2(C[a][r], C[a][r + 1]);
+      fwht8x2(v);
 #pragma unroll
-      for (int a = 0; a < 8; ++a) R[(ntl * 8 + a) * 4 + r] = v[a];
+      for (int a = 0; a < 8; ++a) {
+        R[(ntl * 8 + a) * 4 + r] = v[a].x;
+        R[(ntl * 8 + a) * 4 + r + 1] = v[a].y;
+      }
     }
   }
 }
@@ -167,35 +199,20 @@ __device__ __forceinline__ void rotate_v(const QuantSmem& sm, int warp, int lane
 // ---------------------------------------------------------------- the tile
 
 template <int SIDE, int BITS>
-__device__ __forceinline__ void quantize_tile(const QuantArgs& p, QuantSmem& sm, int64_t grp, int h) {
+__device__ __forceinline__ void quantize_tile(const QuantArgs& p, QuantSmem& sm, uint32_t xs, int64_t grp, int h,
+                                              int64_t blk) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, c = lane & 3;
 
-  // which paged block: slot_mapping[128 * grp] must start a block of the pool
-  const int64_t slot = p.slot_mapping[grp * kTile];
-  const int64_t blk = slot >> 7;
-  if (slot < 0 || (slot & 127) != 0 || blk >= p.num_blocks) {
-    if (tid == 0) report_status(p.status, KVARN_DEV_BAD_SLOT);
-    return;
-  }
-
-  // ---- 1. stage the fp16 tile
-  const __half* src = (SIDE == 0 ? p.k : p.v) + (grp * kTile * p.hkv + h) * (int64_t)kHeadDim;
-  const int64_t row_stride = (int64_t)p.hkv * kHeadDim;
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const int idx = i * kQThreads + tid;
-    const int t = idx >> 4, ch = idx & 15;
-    const uint4 val = __ldg(reinterpret_cast<const uint4*>(src + t * row_stride + ch * 8));
-    *reinterpret_cast<uint4*>(sm.x + t * 256 + ((ch ^ (t & 7)) << 4)) = val;
-  }
-  __syncthreads();
-
   // ---- 2. rotate
   float A[128];
-  if (SIDE == 0) rotate_k(sm, warp, lane, A); else rotate_v(sm, warp, lane, A);
+  if (SIDE == 0) rotate_k(xs, warp, lane, A); else rotate_v(xs, warp, lane, A);
 #pragma unroll
-  for (int i = 0; i < 128; ++i) A[i] = A[i] * A[i];
+  for (int i = 0; i < 128; i += 2) {
+    const float2 s2 = __fmul2_rn(f2(A[i], A[i + 1]), f2(A[i], A[i + 1]));
+    A[i] = s2.x;
+    A[i + 1] = s2.y;
+  }
 
   // ---- 3. normalise
   constexpr int NT = SIDE == 0 ? 4 : 8;   // tokens per thread
@@ -211,37 +228,37 @@ __device__ __forceinline__ void quantize_tile(const QuantArgs& p, QuantSmem& sm,
 #pragma unroll
       for (int a = 0; a < 8; ++a)
 #pragma unroll
-        for (int nb = 0; nb < 2; ++nb)
+        for (int nb = 0; nb < 2; ++nb) {
+          float2 acc = f2(0.f, 0.f);
 #pragma unroll
-          for (int rj = 0; rj < 2; ++rj) {
-            float acc = 0.f;
+          for (int ml = 0; ml < 2; ++ml)
 #pragma unroll
-            for (int ml = 0; ml < 2; ++ml)
-#pragma unroll
-              for (int ri = 0; ri < 2; ++ri)
-                acc = fmaf(A[((ml * 8 + a) * 2 + nb) * 4 + 2 * ri + rj], wt[ml * 2 + ri], acc);
-            s[a * 4 + nb * 2 + rj] = acc;
-          }
+            for (int ri = 0; ri < 2; ++ri) {
+              const int i = ((ml * 8 + a) * 2 + nb) * 4 + 2 * ri;
+              const float w = wt[ml * 2 + ri];
+              acc = __ffma2_rn(f2(A[i], A[i + 1]), f2(w, w), acc);
+            }
+          s[a * 4 + nb * 2] = acc.x;
+          s[a * 4 + nb * 2 + 1] = acc.y;
+        }
       rs_step<32>(s, 16, lane);
       rs_step<16>(s, 8, lane);
       rs_step<8>(s, 4, lane);
-#pragma unroll
-      for (int nb = 0; nb < 2; ++nb)
-#pragma unroll
-        for (int rj = 0; rj < 2; ++rj) sm.red[warp][16 * g + 8 * nb + 2 * c + rj] = s[nb * 2 + rj];
+      *reinterpret_cast<float2*>(&sm.red[warp][16 * g + 2 * c]) = f2(s[0], s[1]);
+      *reinterpret_cast<float2*>(&sm.red[warp][16 * g + 8 + 2 * c]) = f2(s[2], s[3]);
     } else {
       float s[16];   // index a*2 + ri
 #pragma unroll
       for (int a = 0; a < 8; ++a)
 #pragma unroll
         for (int ri = 0; ri < 2; ++ri) {
-          float acc = 0.f;
+          float2 acc = f2(0.f, 0.f);
 #pragma unroll
-          for (int ntl = 0; ntl < 4; ++ntl)
-#pragma unroll
-            for (int rj = 0; rj < 2; ++rj)
-              acc = fmaf(A[(ntl * 8 + a) * 4 + 2 * ri + rj], wt[ntl * 2 + rj], acc);
-          s[a * 2 + ri] = acc;
+          for (int ntl = 0; ntl < 4; ++ntl) {
+            const int i = (ntl * 8 + a) * 4 + 2 * ri;
+            acc = __ffma2_rn(f2(A[i], A[i + 1]), f2(wt[ntl * 2], wt[ntl * 2 + 1]), acc);
+          }
+          s[a * 2 + ri] = acc.x + acc.y;
         }
       rs_step<16>(s, 2, lane);
       rs_step<8>(s, 1, lane);
@@ -253,42 +270,41 @@ __device__ __forceinline__ void quantize_tile(const QuantArgs& p, QuantSmem& sm,
     }
     __syncthreads();
     {
-      const float tot = sm.red[0][tid] + sm.red[1][tid] + sm.red[2][tid] + sm.red[3][tid];
+      const float tot = (sm.red[0][tid] + sm.red[1][tid]) + (sm.red[2][tid] + sm.red[3][tid]);
       lc_own = log2_scale(tot);
-      sm.u[tid] = exp2f(-2.f * lc_own);
+      sm.u[tid] = ex2_fast(-2.f * lc_own);
     }
     __syncthreads();
 
     // token pass
     if (SIDE == 0) {
-      float uu[32];
+      float2 uu[16];   // (a, nb) -> channels 16a + 8nb + 2c + {0,1}
 #pragma unroll
       for (int a = 0; a < 8; ++a)
 #pragma unroll
-        for (int nb = 0; nb < 2; ++nb) {
-          const float2 v2 = *reinterpret_cast<const float2*>(&sm.u[16 * a + 8 * nb + 2 * c]);
-          uu[a * 4 + nb * 2] = v2.x;
-          uu[a * 4 + nb * 2 + 1] = v2.y;
-        }
+        for (int nb = 0; nb < 2; ++nb)
+          uu[a * 2 + nb] = *reinterpret_cast<const float2*>(&sm.u[16 * a + 8 * nb + 2 * c]);
       float s[4];    // index ml*2 + ri
 #pragma unroll
       for (int ml = 0; ml < 2; ++ml)
 #pragma unroll
         for (int ri = 0; ri < 2; ++ri) {
-          float acc = 0.f;
+          float2 acc[4] = {f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f)};   // 4 chains for ILP
 #pragma unroll
           for (int a = 0; a < 8; ++a)
 #pragma unroll
-            for (int nb = 0; nb < 2; ++nb)
-#pragma unroll
-              for (int rj = 0; rj < 2; ++rj)
-                acc = fmaf(A[((ml * 8 + a) * 2 + nb) * 4 + 2 * ri + rj], uu[a * 4 + nb * 2 + rj], acc);
-          s[ml * 2 + ri] = acc;
+            for (int nb = 0; nb < 2; ++nb) {
+              const int i = ((ml * 8 + a) * 2 + nb) * 4 + 2 * ri;
+              acc[(a & 1) * 2 + nb] = __ffma2_rn(f2(A[i], A[i + 1]), uu[a * 2 + nb], acc[(a & 1) * 2 + nb]);
+            }
+          const float2 t01 = __fadd2_rn(acc[0], acc[1]), t23 = __fadd2_rn(acc[2], acc[3]);
+          const float2 t = __fadd2_rn(t01, t23);
+          s[ml * 2 + ri] = t.x + t.y;
         }
       rs_step<4>(s, 2, lane);
       rs_step<2>(s, 1, lane);
       lt_own = log2_scale(s[0]);
-      const float wown = exp2f(-2.f * lt_own);
+      const float wown = ex2_fast(-2.f * lt_own);
 #pragma unroll
       for (int k = 0; k < 4; ++k) wt[k] = __shfl_sync(0xffffffffu, wown, (lane & ~3) | k);
     } else {
@@ -299,22 +315,25 @@ __device__ __forceinline__ void quantize_tile(const QuantArgs& p, QuantSmem& sm,
         for (int ri = 0; ri < 2; ++ri) uu[a * 2 + ri] = sm.u[16 * a + g + 8 * ri];
       float s[8];    // index ntl*2 + rj
 #pragma unroll
-      for (int ntl = 0; ntl < 4; ++ntl)
+      for (int ntl = 0; ntl < 4; ++ntl) {
+        float2 acc[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};   // 2 chains for ILP
 #pragma unroll
-        for (int rj = 0; rj < 2; ++rj) {
-          float acc = 0.f;
+        for (int a = 0; a < 8; ++a)
 #pragma unroll
-          for (int a = 0; a < 8; ++a)
-#pragma unroll
-            for (int ri = 0; ri < 2; ++ri)
-              acc = fmaf(A[(ntl * 8 + a) * 4 + 2 * ri + rj], uu[a * 2 + ri], acc);
-          s[ntl * 2 + rj] = acc;
-        }
+          for (int ri = 0; ri < 2; ++ri) {
+            const int i = (ntl * 8 + a) * 4 + 2 * ri;
+            const float uv = uu[a * 2 + ri];
+            acc[ri] = __ffma2_rn(f2(A[i], A[i + 1]), f2(uv, uv), acc[ri]);
+          }
+        const float2 t = __fadd2_rn(acc[0], acc[1]);
+        s[ntl * 2] = t.x;
+        s[ntl * 2 + 1] = t.y;
+      }
       rs_step<8>(s, 16, lane);
       rs_step<4>(s, 8, lane);
       rs_step<2>(s, 4, lane);
       lt_own = log2_scale(s[0]);
-      const float wown = exp2f(-2.f * lt_own);
+      const float wown = ex2_fast(-2.f * lt_own);
 #pragma unroll
       for (int k = 0; k < 8; ++k) wt[k] = __shfl_sync(0xffffffffu, wown, c | (k << 2));
     }
@@ -338,8 +357,8 @@ __device__ __forceinline__ void quantize_tile(const QuantArgs& p, QuantSmem& sm,
 
   // ---- 4. quantise: recompute R (same arithmetic), Z, zero/step, codes
   float Z[128];
-  if (SIDE == 0) rotate_k(sm, warp, lane, Z); else rotate_v(sm, warp, lane, Z);
-  float zlo = 3.402823466e38f, zhi = -3.402823466e38f;
+  if (SIDE == 0) rotate_k(xs, warp, lane, Z); else rotate_v(xs, warp, lane, Z);
+  float2 zlo = f2(3.402823466e38f, 3.402823466e38f), zhi = f2(-3.402823466e38f, -3.402823466e38f);
   if (SIDE == 0) {
     float mtv[4];
 #pragma unroll
@@ -354,44 +373,41 @@ __device__ __forceinline__ void quantize_tile(const QuantArgs& p, QuantSmem& sm,
 #pragma unroll
         for (int ml = 0; ml < 2; ++ml)
 #pragma unroll
-          for (int ri = 0; ri < 2; ++ri)
-#pragma unroll
-            for (int rj = 0; rj < 2; ++rj) {
-              float& z = Z[((ml * 8 + a) * 2 + nb) * 4 + 2 * ri + rj];
-              z = __fmul_rn(__fmul_rn(z, mtv[ml * 2 + ri]), rj ? mc2.y : mc2.x);
-              zlo = fminf(zlo, z);
-              zhi = fmaxf(zhi, z);
-            }
+          for (int ri = 0; ri < 2; ++ri) {
+            const int i = ((ml * 8 + a) * 2 + nb) * 4 + 2 * ri;
+            const float m = mtv[ml * 2 + ri];
+            const float2 z = __fmul2_rn(__fmul2_rn(f2(Z[i], Z[i + 1]), f2(m, m)), mc2);
+            Z[i] = z.x;
+            Z[i + 1] = z.y;
+            zlo = f2(fminf(zlo.x, z.x), fminf(zlo.y, z.y));
+            zhi = f2(fmaxf(zhi.x, z.x), fmaxf(zhi.y, z.y));
+          }
       }
   } else {
-    float mtv[8];
+    float2 mtv[4];
 #pragma unroll
-    for (int ntl = 0; ntl < 4; ++ntl) {
-      const float2 m2 = *reinterpret_cast<const float2*>(&sm.mt[8 * (4 * warp + ntl) + 2 * c]);
-      mtv[ntl * 2] = m2.x;
-      mtv[ntl * 2 + 1] = m2.y;
-    }
+    for (int ntl = 0; ntl < 4; ++ntl) mtv[ntl] = *reinterpret_cast<const float2*>(&sm.mt[8 * (4 * warp + ntl) + 2 * c]);
 #pragma unroll
     for (int a = 0; a < 8; ++a)
 #pragma unroll
       for (int ri = 0; ri < 2; ++ri) {
         const float mcv = sm.mc[16 * a + g + 8 * ri];
 #pragma unroll
-        for (int ntl = 0; ntl < 4; ++ntl)
-#pragma unroll
-          for (int rj = 0; rj < 2; ++rj) {
-            float& z = Z[(ntl * 8 + a) * 4 + 2 * ri + rj];
-            z = __fmul_rn(__fmul_rn(z, mtv[ntl * 2 + rj]), mcv);
-            zlo = fminf(zlo, z);
-            zhi = fmaxf(zhi, z);
-          }
+        for (int ntl = 0; ntl < 4; ++ntl) {
+          const int i = (ntl * 8 + a) * 4 + 2 * ri;
+          const float2 z = __fmul2_rn(__fmul2_rn(f2(Z[i], Z[i + 1]), mtv[ntl]), f2(mcv, mcv));
+          Z[i] = z.x;
+          Z[i + 1] = z.y;
+          zlo = f2(fminf(zlo.x, z.x), fminf(zlo.y, z.y));
+          zhi = f2(fmaxf(zhi.x, z.x), fmaxf(zhi.y, z.y));
+        }
       }
   }
-  zlo = warp_min(zlo);
-  zhi = warp_max(zhi);
+  const float zl = warp_min(fminf(zlo.x, zlo.y));
+  const float zh = warp_max(fmaxf(zhi.x, zhi.y));
   if (lane == 0) {
-    sm.zmin[warp] = zlo;
-    sm.zmax[warp] = zhi;
+    sm.zmin[warp] = zl;
+    sm.zmax[warp] = zh;
   }
   __syncthreads();
   const float zero = fminf(fminf(sm.zmin[0], sm.zmin[1]), fminf(sm.zmin[2], sm.zmin[3]));
@@ -401,31 +417,33 @@ __device__ __forceinline__ void quantize_tile(const QuantArgs& p, QuantSmem& sm,
   if (step == 0.f) step = 1.f;
   const float inv = __fdiv_rn(1.f, step);
 
-  // codes, packed in the fragment order: block-local index bl (0..15), register j, half h
+  // codes: y = (Z - zero) * inv >= 0, rounded to nearest even by adding 1.5 * 2^23
+  // (exact for y < 2^22); packed in the fragment order (block bl, register j, half h)
   constexpr int PER = 16 / BITS;          // register pairs per 32-bit word
   constexpr int NW = 64 / PER;            // words per thread (= 4*BITS)
+  constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23
   uint32_t words[NW];
 #pragma unroll
   for (int i = 0; i < NW; ++i) words[i] = 0u;
 #pragma unroll
   for (int bl = 0; bl < 16; ++bl)
 #pragma unroll
-    for (int j = 0; j < 4; ++j)
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        int idx;
-        if (SIDE == 0) {   // bl = ml*8 + a;  j = ri + 2*nb;  h = rj
-          const int ml = bl >> 3, a = bl & 7, nb = j >> 1, ri = j & 1;
-          idx = ((ml * 8 + a) * 2 + nb) * 4 + 2 * ri + hh;
-        } else {           // bl = (ntl>>1)*8 + a;  j = ri + 2*(ntl&1);  h = rj
-          const int ntl = 2 * (bl >> 3) + (j >> 1), a = bl & 7, ri = j & 1;
-          idx = (ntl * 8 + a) * 4 + 2 * ri + hh;
-        }
-        const float y = __fmul_rn(__fsub_rn(Z[idx], zero), inv);
-        const int code = min(max(__float2int_rn(y), 0), LB);
-        const int rho = 4 * bl + j;
-        words[rho / PER] |= static_cast<uint32_t>(code) << (BITS * (rho % PER) + 16 * hh);
+    for (int j = 0; j < 4; ++j) {
+      int idx;                             // index of the (h = 0) element; h = 1 is idx + 1
+      if (SIDE == 0) {   // bl = ml*8 + a;  j = ri + 2*nb;  h = rj
+        const int ml = bl >> 3, a = bl & 7, nb = j >> 1, ri = j & 1;
+        idx = ((ml * 8 + a) * 2 + nb) * 4 + 2 * ri;
+      } else {           // bl = (ntl>>1)*8 + a;  j = ri + 2*(ntl&1);  h = rj
+        const int ntl = 2 * (bl >> 3) + (j >> 1), a = bl & 7, ri = j & 1;
+        idx = (ntl * 8 + a) * 4 + 2 * ri;
       }
+      const float2 y = __fmul2_rn(__fadd2_rn(f2(Z[idx], Z[idx + 1]), f2(-zero, -zero)), f2(inv, inv));
+      const float2 r = __fadd2_rn(y, f2(kMagic, kMagic));
+      // 0 <= y <= 2^b - 1 up to rounding, so rne(y) sits in the low BITS bits of r
+      const int rho = 4 * bl + j;
+      words[rho / PER] = bfi(__float_as_uint(r.x), words[rho / PER], BITS * (rho % PER), BITS);
+      words[rho / PER] = bfi(__float_as_uint(r.y), words[rho / PER], BITS * (rho % PER) + 16, BITS);
+    }
 
   // ---- 5. store codes (16-byte chunks, lane-interleaved) and the scale record
   uint8_t* dst = p.packed + (blk * p.hkv + h) * (int64_t)(2048 * (p.kb + p.vb)) + (SIDE == 0 ? 0 : 2048 * p.kb);
@@ -448,19 +466,147 @@ __device__ __forceinline__ void quantize_tile(const QuantArgs& p, QuantSmem& sm,
   }
 }
 
+// TMA load of one tile (two 64-channel boxes) into a stage
+__device__ __forceinline__ void load_tile(const CUtensorMap* map, uint8_t* dst, uint64_t* bar, int h, int64_t grp) {
+  mbar_arrive_expect_tx(bar, 2 * kBox);
+  const int t0 = static_cast<int>(grp * kTile);
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];\n" ::"r"(smem_u32(dst + half * kBox)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(64 * half), "r"(h), "r"(t0), "r"(smem_u32(bar))
+        : "memory");
+  }
+}
+
 template <int KB, int VB>
-__global__ void __launch_bounds__(kQThreads) quantize_kernel(QuantArgs p) {
-  __shared__ QuantSmem sm;
-  const int64_t grp = blockIdx.x;
-  const int h = blockIdx.y;
-  if (blockIdx.z == 0) quantize_tile<0, KB>(p, sm, grp, h);
-  else quantize_tile<1, VB>(p, sm, grp, h);
+#ifndef KVARN_Q_MIN_CTAS
+#define KVARN_Q_MIN_CTAS 3
+#endif
+__global__ void __launch_bounds__(kQThreads, KVARN_Q_MIN_CTAS) quantize_kernel(const __grid_constant__ CUtensorMap map_k,
+                                                            const __grid_constant__ CUtensorMap map_v,
+                                                            const QuantArgs p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  QuantSmem& sm = *reinterpret_cast<QuantSmem*>(smem_raw);
+  const int tid = threadIdx.x;
+  const int64_t per_side = p.num_groups * p.hkv;
+  const int64_t total = 2 * per_side;
+  // tile id -> (side, group, head): K tiles first, then V tiles
+  auto decode_id = [&](int64_t id, int& side, int64_t& grp, int& h) {
+    side = id >= per_side ? 1 : 0;
+    const int64_t r = id - side * per_side;
+    grp = r / p.hkv;
+    h = static_cast<int>(r - grp * p.hkv);
+  };
+  if (tid == 0) {
+    mbar_init(&sm.bar[0], 1);
+    mbar_init(&sm.bar[1], 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  int64_t id = blockIdx.x;
+  if (id < total && tid == 0) {
+    int side, h;
+    int64_t grp;
+    decode_id(id, side, grp, h);
+    load_tile(side ? &map_v : &map_k, sm.x[0][0], &sm.bar[0], h, grp);
+  }
+  for (int it = 0; id < total; ++it, id += gridDim.x) {
+    const int stage = it & 1;
+    const int64_t nxt = id + gridDim.x;
+    if (nxt < total && tid == 0) {   // the other stage was released at the end of the previous tile
+      int side, h;
+      int64_t grp;
+      decode_id(nxt, side, grp, h);
+      load_tile(side ? &map_v : &map_k, sm.x[stage ^ 1][0], &sm.bar[stage ^ 1], h, grp);
+    }
+    int side, h;
+    int64_t grp;
+    decode_id(id, side, grp, h);
+    // every thread polls; the CTA proceeds only if all saw the copy land
+    const bool landed = __syncthreads_and(mbar_wait_bounded(&sm.bar[stage], (it >> 1) & 1)) != 0;
+    if (!landed) {
+      if (tid == 0) report_status(p.status, KVARN_DEV_TIMEOUT);
+      // let the copies still in flight land before the shared memory is released
+      (void)mbar_wait_bounded(&sm.bar[stage], (it >> 1) & 1);
+      if (nxt < total) (void)mbar_wait_bounded(&sm.bar[stage ^ 1], ((it + 1) >> 1) & 1);
+      return;
+    }
+    // which paged block: slot_mapping[128 * grp] must start a block of the pool
+    const int64_t slot = p.slot_mapping[grp * kTile];
+    const int64_t blk = slot >> 7;
+    if (slot < 0 || (slot & 127) != 0 || blk >= p.num_blocks) {
+      if (tid == 0) report_status(p.status, KVARN_DEV_BAD_SLOT);
+    } else {
+      const uint32_t xs = smem_u32(sm.x[stage][0]);
+      if (side == 0) quantize_tile<0, KB>(p, sm, xs, grp, h, blk);
+      else quantize_tile<1, VB>(p, sm, xs, grp, h, blk);
+    }
+    __syncthreads();   // stage `stage` and the shared scratch are free again
+  }
+}
+
+// ---------------------------------------------------------------- host side
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static std::once_flag once;
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+// [num_tokens][hkv][128] fp16 as a 3-D tensor (channel, head, token); box = 64 channels x 1 head x 128 tokens
+cudaError_t make_map(CUtensorMap* m, const __half* base, int hkv, int64_t num_tokens) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (enc == nullptr) return cudaErrorNotSupported;
+  const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(hkv), static_cast<cuuint64_t>(num_tokens)};
+  const cuuint64_t strides[2] = {256, static_cast<cuuint64_t>(hkv) * 256};
+  const cuuint32_t box[3] = {64, 1, 128};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<__half*>(base), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
 template <int KB, int VB>
 cudaError_t launch_q(const QuantArgs& p, cudaStream_t stream) {
-  const dim3 grid(static_cast<unsigned>(p.num_groups), static_cast<unsigned>(p.hkv), 2);
-  quantize_kernel<KB, VB><<<grid, kQThreads, 0, stream>>>(p);
+  static std::atomic<uint64_t> configured{0};   // one bit per device ordinal
+  static int ctas_per_sm[64] = {};
+  static int sms[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = 1ull << (dev & 63);
+  const int smem = static_cast<int>(sizeof(QuantSmem));
+  if ((configured.load(std::memory_order_acquire) & bit) == 0) {
+    e = cudaFuncSetAttribute(quantize_kernel<KB, VB>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    int occ = 0, n = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, quantize_kernel<KB, VB>, kQThreads, smem);
+    if (e != cudaSuccess) return e;
+    e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    ctas_per_sm[dev & 63] = occ > 0 ? occ : 1;
+    sms[dev & 63] = n;
+    configured.fetch_or(bit, std::memory_order_acq_rel);
+  }
+  CUtensorMap mk, mv;
+  e = make_map(&mk, p.k, p.hkv, p.num_groups * kTile);
+  if (e != cudaSuccess) return e;
+  e = make_map(&mv, p.v, p.hkv, p.num_groups * kTile);
+  if (e != cudaSuccess) return e;
+  const int64_t tiles = 2 * p.num_groups * p.hkv;
+  const int64_t slots = static_cast<int64_t>(sms[dev & 63]) * ctas_per_sm[dev & 63];
+  const unsigned grid = static_cast<unsigned>(tiles < slots ? tiles : slots);
+  quantize_kernel<KB, VB><<<grid, kQThreads, smem, stream>>>(mk, mv, p);
   return cudaGetLastError();
 }
 

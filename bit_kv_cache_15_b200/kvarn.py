@@ -190,8 +190,8 @@ def decode_attention(q: torch.Tensor, packed_cache: torch.Tensor, scales: torch.
     d = dims(B, Hq, Hkv, int(block_table.shape[1]), int(packed_cache.shape[0]))
     if out is None:
         out = torch.empty_like(q)
-    if workspace is None:
-        workspace = torch.empty(decode_workspace_bytes(cfg, d), dtype=torch.uint8, device=q.device)
+    if workspace is None:   # zeroed: the trailing arrival counters must start at zero
+        workspace = torch.zeros(decode_workspace_bytes(cfg, d), dtype=torch.uint8, device=q.device)
     st = _lib.kvarn_decode_attention(_ptr(q), _ptr(packed_cache), _ptr(scales), _ptr(fp16_tail), _ptr(block_table),
                                      _ptr(seq_lens), _ptr(out), ctypes.byref(d), ctypes.byref(cfg),
                                      _ptr(workspace), workspace.numel() * workspace.element_size(),
@@ -233,7 +233,7 @@ def decode_attention_fp16(q, k_cache, v_cache, block_table, seq_lens, out=None, 
     d = dims(B, Hq, int(k_cache.shape[1]), int(block_table.shape[1]), int(k_cache.shape[0]))
     out = torch.empty_like(q) if out is None else out
     if workspace is None:
-        workspace = torch.empty(baseline_workspace_bytes(d), dtype=torch.uint8, device=q.device)
+        workspace = torch.zeros(baseline_workspace_bytes(d), dtype=torch.uint8, device=q.device)
     st = _lib.kvarn_decode_attention_fp16(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(seq_lens),
                                           _ptr(out), ctypes.byref(d), sm_scale, _ptr(workspace),
                                           workspace.numel() * workspace.element_size(), _ptr(dev_status),
@@ -252,7 +252,7 @@ def decode_attention_fp8(q, k_cache, v_cache, block_table, seq_lens, k_scale, v_
     d = dims(B, Hq, int(k_cache.shape[1]), int(block_table.shape[1]), int(k_cache.shape[0]))
     out = torch.empty_like(q) if out is None else out
     if workspace is None:
-        workspace = torch.empty(baseline_workspace_bytes(d), dtype=torch.uint8, device=q.device)
+        workspace = torch.zeros(baseline_workspace_bytes(d), dtype=torch.uint8, device=q.device)
     st = _lib.kvarn_decode_attention_fp8(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(seq_lens),
                                          _ptr(out), ctypes.byref(d), sm_scale, k_scale, v_scale, _ptr(workspace),
                                          workspace.numel() * workspace.element_size(), _ptr(dev_status),

@@ -104,8 +104,10 @@ KVARN_API size_t kvarn_cache_bytes_per_block(const kvarn_config* cfg, int32_t nu
 /* Bytes of scales per paged block: num_kv_heads * 2 * 528. */
 KVARN_API size_t kvarn_scale_bytes_per_block(int32_t num_kv_heads);
 
-/* Bytes of decode workspace needed for these dims (the split-K partials).
- * Depends only on cfg and dims (not on seq_lens or the device). */
+/* Bytes of decode workspace needed for these dims: the split-K partial
+ * records followed by one int32 arrival counter per (sequence, KV head).
+ * Depends only on cfg and dims (not on seq_lens or the device).  Its
+ * contents need no initialisation: each call clears its counters first. */
 KVARN_API size_t kvarn_decode_workspace_bytes(const kvarn_config* cfg, const kvarn_decode_dims* dims);
 
 /* Quantise-on-write of whole 128-token tiles ([hypho] 四步流水线 steps 1-4;
@@ -151,7 +153,8 @@ KVARN_API kvarn_status kvarn_quantize_tiles_debug(const void* k, const void* v, 
  *               only; the host never synchronises).
  *  out          fp16 [B][Hq][128]; sequence b, q head j attends with KV head
  *               j / (Hq/Hkv).  A zero-length sequence gets 0.
- *  workspace    device scratch of at least kvarn_decode_workspace_bytes().
+ *  workspace    device scratch of at least kvarn_decode_workspace_bytes();
+ *               calls that share a workspace must not overlap on the GPU.
  * Key side: q H is multiplied by the per-channel scales, the per-token scales
  * multiply the scores; value side: the per-token scales multiply the softmax
  * weights, the per-channel scales and H/128 apply to the output. */
@@ -181,10 +184,12 @@ KVARN_API kvarn_status kvarn_decode_attention(const void* q, const void* packed_
  *    (cudaGetSymbolAddress) with that device current and caches it; make that
  *    first call before any stream capture begins.
  *  - All calls on a device share the one array and it keeps the previous
- *    call's contents.  Nothing in it needs to start at zero: every record a
- *    call reads was written earlier in the same call.  Calls whose kernels
- *    overlap on the GPU (different streams, no ordering) race on the array;
- *    order them on one stream or by events.
+ *    call's contents.  The only words that must start at zero are the
+ *    per-(sequence, KV head) arrival counters, and each call clears them
+ *    (cudaMemsetAsync on the array, no allocation) before its kernel runs;
+ *    the partial records a call reads are written earlier in the same call.
+ *    Calls whose kernels overlap on the GPU (different streams, no ordering)
+ *    race on the array; order them on one stream or by events.
  *  - It calls no cudaMalloc, cudaFree or other allocating routine. */
 KVARN_API kvarn_status kvarn_decode_attention_noalloc(const void* q, const void* packed_cache, const void* scales,
                                                       const void* fp16_tail, const int32_t* block_table,
