@@ -301,12 +301,93 @@ def run_gpu(args):
             },
             "clocks": clocks,
         }
+        if world == 1 and not args.no_sweep:
+            line["sweep"] = {"workload": "decode only, batch 8 at 16384 + ragged tail, Hq=64 Hkv=8, L2 flushed "
+                                         "before each call", "results": precision_sweep(w, dev)}
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(w, rows, budget_s=args.cpu_budget)
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+# ------------------------------------------------------------------ precision sweep (outside the timed step)
+
+def precision_sweep(w, dev, iters=30):
+    """Decode-only time of the same batch-8 16K (+tail) problem at k8v8 / k4v4 /
+    k4v2 / k2v2 and over uncompressed fp16 and e4m3 caches (the in-library
+    baselines).  Each call is timed alone with CUDA events after a 256 MB write
+    that flushes L2.  Returns {name: {us, tokens_per_s, hbm_gbs, bytes}}."""
+    import torch
+    from bit_kv_cache_15_b200 import kvarn as K
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    q = torch.from_numpy(w.q).to(dev)
+    tail = torch.from_numpy(w.tail).to(dev)
+    bt = torch.from_numpy(w.block_table).to(dev)
+    sl = torch.from_numpy(w.seq_lens).to(dev)
+    out = torch.empty_like(q)
+    lens = [int(x) for x in w.seq_lens]
+    n_full_tok = sum(L // 128 * 128 for L in lens)
+    tail_tok = sum(L % 128 for L in lens)
+    res = {}
+
+    def timed(fn):
+        fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(iters):
+            flush.fill_(1)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        return statistics.median(ts) * 1e3
+
+    kf = torch.from_numpy(w.k_full).to(dev)
+    vf = torch.from_numpy(w.v_full).to(dev)
+    slot = torch.from_numpy(w.slot_mapping).to(dev)
+    for kb, vb in ((8, 8), (4, 4), (4, 2), (2, 2)):
+        cfg = K.config(f"kvarn_k{kb}v{vb}_g128")
+        packed, scales = K.alloc_cache(cfg, w.num_blocks, HKV, device=dev)
+        K.quantize_tiles(kf, vf, slot, packed, scales, cfg)
+        d = K.dims(BATCH, HQ, HKV, w.max_blocks_per_seq, w.num_blocks)
+        ws = torch.empty(K.decode_workspace_bytes(cfg, d), dtype=torch.uint8, device=dev)
+        us = timed(lambda: K.decode_attention(q, packed, scales, tail, bt, sl, cfg, out=out, workspace=ws))
+        nbytes = HKV * (n_full_tok // 128 * (2048 * (kb + vb) + 1056) + tail_tok * 512) + 2 * BATCH * HQ * 256
+        res[f"k{kb}v{vb}"] = {"us": us, "tokens_per_s": BATCH / (us * 1e-6), "hbm_gbs": nbytes / (us * 1e-6) / 1e9,
+                              "bytes": nbytes}
+        del packed, scales
+    # uncompressed caches: full tiles from the same K/V, the tail in one extra block per sequence
+    nb = w.num_blocks + BATCH
+    kc = torch.zeros((nb, HKV, 128, 128), dtype=torch.float16, device=dev)
+    vc = torch.zeros_like(kc)
+    blk = torch.from_numpy(w.slot_mapping[::128] // 128).to(dev)
+    kc[blk] = kf.view(-1, 128, HKV, 128).transpose(1, 2)
+    vc[blk] = vf.view(-1, 128, HKV, 128).transpose(1, 2)
+    bt2 = w.block_table.copy()
+    for b, L in enumerate(lens):
+        if L % 128:
+            bt2[b, L // 128] = w.num_blocks + b
+            kc[w.num_blocks + b] = tail[b, 0]
+            vc[w.num_blocks + b] = tail[b, 1]
+    bt2d = torch.from_numpy(bt2).to(dev)
+    d = K.dims(BATCH, HQ, HKV, w.max_blocks_per_seq, nb)
+    wsb = torch.empty(K.baseline_workspace_bytes(d), dtype=torch.uint8, device=dev)
+    us = timed(lambda: K.decode_attention_fp16(q, kc, vc, bt2d, sl, out=out, workspace=wsb))
+    nbytes = HKV * (n_full_tok + tail_tok) * 512 + 2 * BATCH * HQ * 256
+    res["fp16"] = {"us": us, "tokens_per_s": BATCH / (us * 1e-6), "hbm_gbs": nbytes / (us * 1e-6) / 1e9, "bytes": nbytes}
+    k_scale = float(kc.abs().max()) / 448.0
+    v_scale = float(vc.abs().max()) / 448.0
+    k8 = (kc.float() / k_scale).to(torch.float8_e4m3fn).view(torch.uint8)
+    v8 = (vc.float() / v_scale).to(torch.float8_e4m3fn).view(torch.uint8)
+    del kc, vc
+    us = timed(lambda: K.decode_attention_fp8(q, k8, v8, bt2d, sl, k_scale, v_scale, out=out, workspace=wsb))
+    nbytes = HKV * (n_full_tok + tail_tok) * 256 + 2 * BATCH * HQ * 256
+    res["fp8"] = {"us": us, "tokens_per_s": BATCH / (us * 1e-6), "hbm_gbs": nbytes / (us * 1e-6) / 1e9, "bytes": nbytes}
+    return res
 
 
 # ------------------------------------------------------------------ the oracle (CPU baseline / reference arm)
@@ -408,6 +489,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -237,6 +237,9 @@ static kvarn_status baseline_impl(const void* q, const void* k_cache, const void
   p.seq_lens = seq_lens;
   p.out = static_cast<__half*>(out);
   p.ws = static_cast<float*>(workspace);
+  p.counters = reinterpret_cast<int*>(static_cast<uint8_t*>(workspace) +
+                                      partial_bytes(dims->num_seqs, dims->num_q_heads, dims->num_kv_heads,
+                                                    dims->max_blocks_per_seq));
   p.B = dims->num_seqs;
   p.Hq = dims->num_q_heads;
   p.Hkv = dims->num_kv_heads;

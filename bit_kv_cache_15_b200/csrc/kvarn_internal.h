@@ -64,7 +64,8 @@ struct BaselineArgs {
   const int32_t* block_table;
   const int32_t* seq_lens;
   __half* out;
-  float* ws;
+  float* ws;            // partial records, then the per-(seq, KV head) counters
+  int* counters;
   int B, Hq, Hkv, G, max_blocks;
   int64_t num_blocks;
   int tiles_per_split, num_splits;
