@@ -341,7 +341,7 @@ __device__ void baseline_combine(const BaselineArgs& p, int b, int h, int L, boo
 template <int FP8>
 __global__ void __launch_bounds__(kBThreads) baseline_kernel(const __grid_constant__ CUtensorMap mk,
                                                              const __grid_constant__ CUtensorMap mv,
-                                                             const BaselineArgs p) {
+                                                             const __grid_constant__ BaselineArgs p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   __shared__ int last_arrival;
   const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;

@@ -33,6 +33,16 @@
 namespace kvarn {
 namespace {
 
+#ifndef KVARN_D_U_SMALL
+#define KVARN_D_U_SMALL 1      // work units per tile when kb + vb <= 6
+#endif
+#ifndef KVARN_D_MIN_CTAS
+#define KVARN_D_MIN_CTAS 2
+#endif
+#ifndef KVARN_D_QR_SMEM
+#define KVARN_D_QR_SMEM 0      // 1: read q H from shared memory per tile instead of holding it in registers
+#endif
+
 constexpr int kDWarps = 4;
 constexpr int kDThreads = 32 * kDWarps;
 constexpr int kDStages = 2;
@@ -45,7 +55,7 @@ struct DecodeTraits {
   static constexpr int kCodeK = 2048 * KB;
   static constexpr int kCodeV = 2048 * VB;
   static constexpr int kCode = kCodeK + kCodeV;
-  static constexpr int U = (KB + VB) <= 6 ? 1 : ((KB + VB) <= 12 ? 2 : 4);
+  static constexpr int U = (KB + VB) <= 6 ? KVARN_D_U_SMALL : ((KB + VB) <= 12 ? 2 : 4);
   static constexpr int MT = 8 / U;                    // 16-token blocks per unit
   static constexpr int kUnitK = kCodeK / U;
   static constexpr int kUnitV = kCodeV / U;
@@ -161,6 +171,32 @@ __device__ void decode_tail(const DecodeArgs& p, uint8_t* smem, float* qs, int b
 
 // ------------------------------------------------------------------ main kernel
 
+// Copy unit `unit` of this warp (physical block blk) into stage k % 2;
+// returns false (and completes the stage's phase empty) for a bad block id.
+template <int KB, int VB>
+__device__ __forceinline__ bool issue_unit(const DecodeArgs& p, uint8_t* stage_base, uint64_t* my_bars, int k,
+                                           int unit, int32_t blk, int h, int lane) {
+  using T = DecodeTraits<KB, VB>;
+  const int part = unit % T::U;
+  const bool ok = blk >= 0 && blk < p.num_blocks;
+  if (lane == 0) {
+    uint8_t* dst = stage_base + (k & 1) * T::kStage;
+    uint64_t* bar = &my_bars[k & 1];
+    if (ok) {
+      const uint8_t* cb = p.packed + ((int64_t)blk * p.Hkv + h) * T::kCode;
+      mbar_arrive_expect_tx(bar, T::kStage);
+      bulk_g2s(dst, cb + part * T::kUnitK, T::kUnitK, bar);
+      bulk_g2s(dst + T::kUnitK, cb + T::kCodeK + part * T::kUnitV, T::kUnitV, bar);
+      bulk_g2s(dst + T::kUnitK + T::kUnitV, p.scales + ((int64_t)blk * p.Hkv + h) * (2 * kScaleRec), 2 * kScaleRec,
+               bar);
+    } else {
+      report_status(p.status, KVARN_DEV_BAD_BLOCK);
+      mbar_arrive_expect_tx(bar, 0);   // completes the phase with no bytes
+    }
+  }
+  return ok;
+}
+
 // One split: tiles [s*T, s*T + T) of sequence b, KV head h; writes one
 // partial record per query head (or nothing if the split is empty).
 template <int KB, int VB>
@@ -234,6 +270,7 @@ __device__ __forceinline__ void decode_split(const DecodeArgs& p, uint8_t* smem,
 
   // ---- per-warp state
   const int g8 = lane >> 2, c = lane & 3;
+#if !KVARN_D_QR_SMEM
   float qr[32];   // q H of head g8 at channels 16kt + 2c + {0,1,8,9}
 #pragma unroll
   for (int kt = 0; kt < 8; ++kt) {
@@ -244,6 +281,7 @@ __device__ __forceinline__ void decode_split(const DecodeArgs& p, uint8_t* smem,
     qr[4 * kt + 2] = hi.x;
     qr[4 * kt + 3] = hi.y;
   }
+#endif
   const float coef0 = p.sm_scale * kLog2e * (1.f / 128.f) * invsig[2 * c];
   const float coef1 = p.sm_scale * kLog2e * (1.f / 128.f) * invsig[2 * c + 1];
   float* scr = reinterpret_cast<float*>(smem + T::kScrOff) + warp * kHeadDim;
@@ -262,36 +300,17 @@ __device__ __forceinline__ void decode_split(const DecodeArgs& p, uint8_t* smem,
   uint64_t* my_bars = bars + warp * kDStages;
   const int32_t* btab = p.block_table + (int64_t)b * p.max_blocks;
 
-  // copy my k-th unit into stage k % 2; false for a bad block id
-  auto issue = [&](int k) {
-    const int unit = warp + k * kDWarps;
-    const int i = t_begin + unit / U, part = unit % U;
-    const int32_t blk = btab[i];
-    const bool ok = blk >= 0 && blk < p.num_blocks;
-    if (lane == 0) {
-      uint8_t* dst = stage_base + (k & 1) * T::kStage;
-      uint64_t* bar = &my_bars[k & 1];
-      if (ok) {
-        const uint8_t* cb = p.packed + ((int64_t)blk * p.Hkv + h) * T::kCode;
-        mbar_arrive_expect_tx(bar, T::kStage);
-        bulk_g2s(dst, cb + part * T::kUnitK, T::kUnitK, bar);
-        bulk_g2s(dst + T::kUnitK, cb + T::kCodeK + part * T::kUnitV, T::kUnitV, bar);
-        bulk_g2s(dst + T::kUnitK + T::kUnitV, p.scales + ((int64_t)blk * p.Hkv + h) * (2 * kScaleRec),
-                 2 * kScaleRec, bar);
-      } else {
-        report_status(p.status, KVARN_DEV_BAD_BLOCK);
-        mbar_arrive_expect_tx(bar, 0);   // completes the phase with no bytes
-      }
-    }
-    return ok;
-  };
-
-  bool ok0 = n_mine > 0 ? issue(0) : false;
-  bool ok1 = n_mine > 1 ? issue(1) : false;
+  bool ok0 = n_mine > 0 ? issue_unit<KB, VB>(p, stage_base, my_bars, 0, warp, btab[t_begin + warp / U], h, lane)
+                        : false;
+  bool ok1 = n_mine > 1 ? issue_unit<KB, VB>(p, stage_base, my_bars, 1, warp + kDWarps,
+                                             btab[t_begin + (warp + kDWarps) / U], h, lane)
+                        : false;
   int k_fail = -1;
 
   for (int k = 0; k < n_mine; ++k) {
     const int stg = k & 1;
+    // block id of unit k + 2, loaded now so it is in hand when that copy is issued
+    const int32_t blk_next = k + 2 < n_mine ? btab[t_begin + (warp + (k + 2) * kDWarps) / U] : 0;
     if (!__all_sync(0xffffffffu, mbar_wait_bounded(&my_bars[stg], (k >> 1) & 1))) {
       if (lane == 0) report_status(p.status, KVARN_DEV_TIMEOUT);
       k_fail = k;
@@ -331,8 +350,15 @@ __device__ __forceinline__ void decode_split(const DecodeArgs& p, uint8_t* smem,
       for (int kt = 0; kt < 8; ++kt) {
         const float2 s01 = *reinterpret_cast<const float2*>(&scr[16 * kt + 2 * c]);
         const float2 s89 = *reinterpret_cast<const float2*>(&scr[16 * kt + 2 * c + 8]);
+#if KVARN_D_QR_SMEM
+        const float2 qlo = *reinterpret_cast<const float2*>(&qrot[g8 * 128 + 16 * kt + 2 * c]);
+        const float2 qhi = *reinterpret_cast<const float2*>(&qrot[g8 * 128 + 16 * kt + 2 * c + 8]);
+        const float x0 = qlo.x * s01.x, x1 = qlo.y * s01.y;
+        const float x8 = qhi.x * s89.x, x9 = qhi.y * s89.y;
+#else
         const float x0 = qr[4 * kt] * s01.x, x1 = qr[4 * kt + 1] * s01.y;
         const float x8 = qr[4 * kt + 2] * s89.x, x9 = qr[4 * kt + 3] * s89.y;
+#endif
         const __half2 h01 = __floats2half2_rn(x0, x1);
         const __half2 h89 = __floats2half2_rn(x8, x9);
         const float2 f01 = __half22float2(h01), f89 = __half22float2(h89);
@@ -479,7 +505,7 @@ __device__ __forceinline__ void decode_split(const DecodeArgs& p, uint8_t* smem,
     }
     __syncwarp();
     if (k + 2 < n_mine) {
-      const bool okn = issue(k + 2);
+      const bool okn = issue_unit<KB, VB>(p, stage_base, my_bars, k + 2, warp + (k + 2) * kDWarps, blk_next, h, lane);
       if (stg == 0) ok0 = okn; else ok1 = okn;
     }
   }
@@ -607,7 +633,7 @@ __device__ void combine_pair(const DecodeArgs& p, int b, int h, int L, bool vali
 // once after its records are visible; the last of the num_splits + 1 arrivals
 // merges them.  Nothing waits on anything.
 template <int KB, int VB>
-__global__ void __launch_bounds__(kDThreads, 2) decode_kernel(const DecodeArgs p) {
+__global__ void __launch_bounds__(kDThreads, KVARN_D_MIN_CTAS) decode_kernel(const __grid_constant__ DecodeArgs p) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ int last_arrival;
   const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;

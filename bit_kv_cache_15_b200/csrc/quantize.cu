@@ -102,6 +102,17 @@ __device__ __forceinline__ void rs_step(float* v, int mask, int lane) {
 
 __device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
 
+__device__ __forceinline__ float min3(float a, float b, float c) {
+  float r;
+  asm("min.f32 %0, %1, %2, %3;\n" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;\n" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 // insert the low `len` bits of x into y at bit `pos`
 __device__ __forceinline__ uint32_t bfi(uint32_t x, uint32_t y, int pos, int len) {
   uint32_t r;
@@ -358,7 +369,7 @@ __device__ __forceinline__ void quantize_tile(const QuantArgs& p, QuantSmem& sm,
   // ---- 4. quantise: recompute R (same arithmetic), Z, zero/step, codes
   float Z[128];
   if (SIDE == 0) rotate_k(xs, warp, lane, Z); else rotate_v(xs, warp, lane, Z);
-  float2 zlo = f2(3.402823466e38f, 3.402823466e38f), zhi = f2(-3.402823466e38f, -3.402823466e38f);
+  float zlo = 3.402823466e38f, zhi = -3.402823466e38f;
   if (SIDE == 0) {
     float mtv[4];
 #pragma unroll
@@ -379,8 +390,8 @@ __device__ __forceinline__ void quantize_tile(const QuantArgs& p, QuantSmem& sm,
             const float2 z = __fmul2_rn(__fmul2_rn(f2(Z[i], Z[i + 1]), f2(m, m)), mc2);
             Z[i] = z.x;
             Z[i + 1] = z.y;
-            zlo = f2(fminf(zlo.x, z.x), fminf(zlo.y, z.y));
-            zhi = f2(fmaxf(zhi.x, z.x), fmaxf(zhi.y, z.y));
+            zlo = min3(zlo, z.x, z.y);
+            zhi = max3(zhi, z.x, z.y);
           }
       }
   } else {
@@ -398,13 +409,13 @@ __device__ __forceinline__ void quantize_tile(const QuantArgs& p, QuantSmem& sm,
           const float2 z = __fmul2_rn(__fmul2_rn(f2(Z[i], Z[i + 1]), mtv[ntl]), f2(mcv, mcv));
           Z[i] = z.x;
           Z[i + 1] = z.y;
-          zlo = f2(fminf(zlo.x, z.x), fminf(zlo.y, z.y));
-          zhi = f2(fmaxf(zhi.x, z.x), fmaxf(zhi.y, z.y));
+          zlo = min3(zlo, z.x, z.y);
+          zhi = max3(zhi, z.x, z.y);
         }
       }
   }
-  const float zl = warp_min(fminf(zlo.x, zlo.y));
-  const float zh = warp_max(fmaxf(zhi.x, zhi.y));
+  const float zl = warp_min(zlo);
+  const float zh = warp_max(zhi);
   if (lane == 0) {
     sm.zmin[warp] = zl;
     sm.zmax[warp] = zh;
@@ -480,25 +491,26 @@ __device__ __forceinline__ void load_tile(const CUtensorMap* map, uint8_t* dst, 
   }
 }
 
+// tile id -> (side, group, head): K tiles first, then V tiles
+__device__ __forceinline__ void tile_coords(const QuantArgs& p, int64_t id, int& side, int64_t& grp, int& h) {
+  const int64_t per_side = p.num_groups * p.hkv;
+  side = id >= per_side ? 1 : 0;
+  const int64_t r = id - side * per_side;
+  grp = r / p.hkv;
+  h = static_cast<int>(r - grp * p.hkv);
+}
+
 template <int KB, int VB>
 #ifndef KVARN_Q_MIN_CTAS
 #define KVARN_Q_MIN_CTAS 3
 #endif
 __global__ void __launch_bounds__(kQThreads, KVARN_Q_MIN_CTAS) quantize_kernel(const __grid_constant__ CUtensorMap map_k,
                                                             const __grid_constant__ CUtensorMap map_v,
-                                                            const QuantArgs p) {
+                                                            const __grid_constant__ QuantArgs p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   QuantSmem& sm = *reinterpret_cast<QuantSmem*>(smem_raw);
   const int tid = threadIdx.x;
-  const int64_t per_side = p.num_groups * p.hkv;
-  const int64_t total = 2 * per_side;
-  // tile id -> (side, group, head): K tiles first, then V tiles
-  auto decode_id = [&](int64_t id, int& side, int64_t& grp, int& h) {
-    side = id >= per_side ? 1 : 0;
-    const int64_t r = id - side * per_side;
-    grp = r / p.hkv;
-    h = static_cast<int>(r - grp * p.hkv);
-  };
+  const int64_t total = 2 * p.num_groups * p.hkv;
   if (tid == 0) {
     mbar_init(&sm.bar[0], 1);
     mbar_init(&sm.bar[1], 1);
@@ -509,7 +521,7 @@ __global__ void __launch_bounds__(kQThreads, KVARN_Q_MIN_CTAS) quantize_kernel(c
   if (id < total && tid == 0) {
     int side, h;
     int64_t grp;
-    decode_id(id, side, grp, h);
+    tile_coords(p, id, side, grp, h);
     load_tile(side ? &map_v : &map_k, sm.x[0][0], &sm.bar[0], h, grp);
   }
   for (int it = 0; id < total; ++it, id += gridDim.x) {
@@ -518,12 +530,12 @@ __global__ void __launch_bounds__(kQThreads, KVARN_Q_MIN_CTAS) quantize_kernel(c
     if (nxt < total && tid == 0) {   // the other stage was released at the end of the previous tile
       int side, h;
       int64_t grp;
-      decode_id(nxt, side, grp, h);
+      tile_coords(p, nxt, side, grp, h);
       load_tile(side ? &map_v : &map_k, sm.x[stage ^ 1][0], &sm.bar[stage ^ 1], h, grp);
     }
     int side, h;
     int64_t grp;
-    decode_id(id, side, grp, h);
+    tile_coords(p, id, side, grp, h);
     // every thread polls; the CTA proceeds only if all saw the copy land
     const bool landed = __syncthreads_and(mbar_wait_bounded(&sm.bar[stage], (it >> 1) & 1)) != 0;
     if (!landed) {
