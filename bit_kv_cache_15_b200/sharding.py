@@ -1,0 +1,36 @@
+"""Data-parallel sharding of the hot path over ranks (one process per GPU).
+
+The path splits into independent units -- quantisation tiles and decode
+(sequence, KV head) problems -- with no exchange step between them, so N
+GPUs each take their own sequences and never communicate on the data path.
+Only the benchmark's timing uses a collective (the max of the per-rank
+elapsed times).
+"""
+from __future__ import annotations
+
+
+def shard_range(global_units: int, rank: int, world: int) -> tuple[int, int]:
+    """Contiguous block of units owned by `rank`: sizes differ by at most one."""
+    if world <= 0 or not 0 <= rank < world:
+        raise ValueError("bad rank / world")
+    base, extra = divmod(global_units, world)
+    start = rank * base + min(rank, extra)
+    return start, start + base + (1 if rank < extra else 0)
+
+
+def rank_seed(seed: int, rank: int) -> int:
+    """Seed of a rank's synthetic batch: distinct per rank, reproducible."""
+    return int(seed) * 1000 + int(rank)
+
+
+def max_over_ranks(value: float, group=None) -> float:
+    """Largest per-rank value (the job's elapsed time), via all_reduce(MAX)."""
+    import torch
+    import torch.distributed as dist
+    if not dist.is_available() or not dist.is_initialized():
+        return float(value)
+    backend = dist.get_backend(group)
+    dev = torch.device("cuda", torch.cuda.current_device()) if backend == "nccl" else torch.device("cpu")
+    t = torch.tensor([float(value)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX, group=group)
+    return float(t.item())
