@@ -70,18 +70,37 @@ struct DecodeTraits {
   static_assert(kDWarps * kDStages * 8 <= 128, "barrier area");
 };
 
+// Where a code of `slot` sits in its fp16 half-word for the mma: bit
+// kBase + kSRow * (slot & 1).  slot & 1 is the fragment row half (channel or
+// token 8..15 of the 16-block) for every width, so the offset factors into a
+// per-row-half power of two with no column-half part.  The positions keep each
+// code in the top bits of the 10-bit mantissa: a subnormal A operand with
+// leading zero mantissa bits costs the tensor core's fp32 accumulation that
+// many bits (it truncates below an alignment point set by the exponent field),
+// and the V-side products, all of one sign, would then sum a coherent bias.
+template <int BITS> struct CodeShift {
+  static constexpr int kBase = BITS == 2 ? 6 : 2;
+  static constexpr int kSRow = BITS == 2 ? 2 : (BITS == 4 ? 4 : 0);
+};
+
 // f16x2 of the two codes in `slot` of a fragment-order word (low half-word:
-// even column, high half-word: odd column), as exact fp16 integers.
+// even column, high half-word: odd column).  The word is shifted so the code
+// lands at its CodeShift position, then masked: with the exponent field zero,
+// each half IS the exact subnormal code * 2^(s - 24).  Slots that share a
+// shift share the shifted word (two distinct shifts per word for 4- and 8-bit
+// codes, four for 2-bit), so a code pair costs one AND plus a shared shift.
 template <int BITS>
-__device__ __forceinline__ uint32_t dequant_slot(uint32_t w, uint32_t w8, int slot) {
-  const int off = BITS * slot;
-  const int s = off & 7;
+__device__ __forceinline__ uint32_t dequant_slot(uint32_t w, int slot) {
+  const int s = CodeShift<BITS>::kBase + CodeShift<BITS>::kSRow * (slot & 1);
+  const int sh = s - BITS * slot;
+  const uint32_t x = sh >= 0 ? (w << sh) : (w >> -sh);
   const uint32_t m1 = ((1u << BITS) - 1u) << s;
-  const uint32_t x = lop_and_or(off >= 8 ? w8 : w, m1 | (m1 << 16), 0x64006400u);
-  const uint32_t sc = static_cast<uint32_t>(15 - s) << 10;           // 2^-s
-  const uint32_t bi = 0x8000u | (static_cast<uint32_t>(25 - s) << 10);  // -1024 * 2^-s
-  return h2_as_u32(__hfma2(u32_as_h2(x), u32_as_h2(sc | (sc << 16)), u32_as_h2(bi | (bi << 16))));
+  return x & (m1 | (m1 << 16));
 }
+
+// Power-of-two boost of the softmax weights fed to the V-side mma (P' <= 2^12,
+// far inside fp16's range, with small weights kept out of the subnormals).
+constexpr int kPBoost = 12;
 
 __device__ __forceinline__ float hf(const __half* p, int i) { return __half2float(p[i]); }
 
@@ -364,12 +383,14 @@ __device__ __forceinline__ void decode_split(const DecodeArgs& p, uint8_t* smem,
         const float2 f01 = __half22float2(h01), f89 = __half22float2(h89);
         const __half2 l01 = __floats2half2_rn(x0 - f01.x, x1 - f01.y);
         const __half2 l89 = __floats2half2_rn(x8 - f89.x, x9 - f89.y);
-        const float2 g01 = __half22float2(l01), g89 = __half22float2(l89);
+        {   // sum of exactly the q' values the mma sees (hi + lo)
+          const float2 g01 = __half22float2(l01), g89 = __half22float2(l89);
+          qsum += ((f01.x + g01.x) + (f01.y + g01.y)) + ((f89.x + g89.x) + (f89.y + g89.y));
+        }
         qb0[kt] = h2_as_u32(h01);
         qb1[kt] = h2_as_u32(h89);
         ql0[kt] = h2_as_u32(l01);
         ql1[kt] = h2_as_u32(l89);
-        qsum += ((f01.x + g01.x) + (f01.y + g01.y)) + ((f89.x + g89.x) + (f89.y + g89.y));
       }
       __syncwarp();   // scr is rewritten by the next unit
       qsum += __shfl_xor_sync(0xffffffffu, qsum, 1);
@@ -395,11 +416,11 @@ __device__ __forceinline__ void decode_split(const DecodeArgs& p, uint8_t* smem,
           const uint32_t wds[4] = {v4.x, v4.y, v4.z, v4.w};
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            const uint32_t w = wds[i], w8 = w >> 8;
+            const uint32_t w = wds[i];
 #pragma unroll
             for (int sl = 0; sl < PK; ++sl) {
               const int rho = (4 * q + i) * PK + sl;
-              afr[rho & 3] = dequant_slot<KB>(w, w8, sl);
+              afr[rho & 3] = dequant_slot<KB>(w, sl);
               if ((rho & 3) == 3) {
                 const int blk = rho >> 2;   // (token block in unit) * 8 + channel block
                 mma_f16(S[blk >> 3], afr[0], afr[1], afr[2], afr[3], qb0[blk & 7], qb1[blk & 7]);
@@ -411,6 +432,9 @@ __device__ __forceinline__ void decode_split(const DecodeArgs& p, uint8_t* smem,
       }
 
       // scores (log2 units) with the token scales, online softmax (a8)
+      // the step with the codes' 2^(s - 24) placement undone, per row half
+      constexpr float kRowK0 = 16777216.f / static_cast<float>(1 << CodeShift<KB>::kBase);
+      constexpr float kRowK1 = kRowK0 / static_cast<float>(1 << CodeShift<KB>::kSRow);
       float tv[MT][2];
       float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
@@ -419,9 +443,10 @@ __device__ __forceinline__ void decode_split(const DecodeArgs& p, uint8_t* smem,
         for (int ri = 0; ri < 2; ++ri) {
           const int t = t0 + 16 * mt + g8 + 8 * ri;
           const float tk = ex2_fast(hf(ltk, t));
-          tv[mt][ri] = ex2_fast(hf(ltv, t));
-          S[mt][2 * ri] = fmaf(sk, S[mt][2 * ri], za0) * (cf0 * tk);
-          S[mt][2 * ri + 1] = fmaf(sk, S[mt][2 * ri + 1], za1) * (cf1 * tk);
+          const float skr = sk * (ri ? kRowK1 : kRowK0);
+          tv[mt][ri] = hf(ltv, t);
+          S[mt][2 * ri] = fmaf(skr, S[mt][2 * ri], za0) * (cf0 * tk);
+          S[mt][2 * ri + 1] = fmaf(skr, S[mt][2 * ri + 1], za1) * (cf1 * tk);
           mx0 = fmaxf(mx0, S[mt][2 * ri]);
           mx1 = fmaxf(mx1, S[mt][2 * ri + 1]);
         }
@@ -430,6 +455,20 @@ __device__ __forceinline__ void decode_split(const DecodeArgs& p, uint8_t* smem,
         mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
         mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
       }
+      // V token scales relative to the tile's largest, times 2^kPBoost: the weights
+      // p * tv fed to the mma then stay in fp16's normal range down to p * tv ~ 2^-26
+      // of the tile maximum; the common factor is undone on the fold below
+      float lvm = tv[0][0];
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt) lvm = fmaxf(lvm, fmaxf(tv[mt][0], tv[mt][1]));
+      lvm = fmaxf(lvm, __shfl_xor_sync(0xffffffffu, lvm, 4));
+      lvm = fmaxf(lvm, __shfl_xor_sync(0xffffffffu, lvm, 8));
+      lvm = fmaxf(lvm, __shfl_xor_sync(0xffffffffu, lvm, 16));
+      lvm = ceilf(lvm);
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+        for (int ri = 0; ri < 2; ++ri) tv[mt][ri] = ex2_fast(tv[mt][ri] - lvm + static_cast<float>(kPBoost));
       const float mn0 = fmaxf(mrun[0], mx0), mn1 = fmaxf(mrun[1], mx1);
       const float al0 = ex2_fast(mrun[0] - mn0), al1 = ex2_fast(mrun[1] - mn1);
       mrun[0] = mn0;
@@ -446,6 +485,8 @@ __device__ __forceinline__ void decode_split(const DecodeArgs& p, uint8_t* smem,
           ls0 += p0;
           ls1 += p1;
           const __half2 hp = __floats2half2_rn(p0 * tv[mt][ri], p1 * tv[mt][ri]);
+          // the zero-point term must use exactly the weights the mma sees: after the
+          // inverse Hadamard a common error across channels lands on one output channel
           const float2 fp = __half22float2(hp);
           ps0 += fp.x;
           ps1 += fp.y;
@@ -478,11 +519,11 @@ __device__ __forceinline__ void decode_split(const DecodeArgs& p, uint8_t* smem,
           const uint32_t wds[4] = {v4.x, v4.y, v4.z, v4.w};
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            const uint32_t w = wds[i], w8 = w >> 8;
+            const uint32_t w = wds[i];
 #pragma unroll
             for (int sl = 0; sl < PV; ++sl) {
               const int rho = (4 * q + i) * PV + sl;
-              afr[rho & 3] = dequant_slot<VB>(w, w8, sl);
+              afr[rho & 3] = dequant_slot<VB>(w, sl);
               if ((rho & 3) == 3) {
                 const int blk = rho >> 2;   // (token block in unit) * 8 + channel block
                 mma_f16(O[blk & 7], afr[0], afr[1], afr[2], afr[3], bv0[blk >> 3], bv1[blk >> 3]);
@@ -493,14 +534,18 @@ __device__ __forceinline__ void decode_split(const DecodeArgs& p, uint8_t* smem,
       }
 
       // fold the V grid and channel scales into the running accumulator
-      const float zp0 = zv * ps0, zp1 = zv * ps1;
+      const float tvf = ex2_fast(lvm - static_cast<float>(kPBoost));
+      const float zp0 = zv * tvf * ps0, zp1 = zv * tvf * ps1;
+      const float sv0 = sv * tvf * (16777216.f / static_cast<float>(1 << CodeShift<VB>::kBase));
+      const float sv1 = sv0 * (1.f / static_cast<float>(1 << CodeShift<VB>::kSRow));
 #pragma unroll
       for (int mt = 0; mt < 8; ++mt)
 #pragma unroll
         for (int ri = 0; ri < 2; ++ri) {
           const float vcs = ex2_fast(hf(lcv, 16 * mt + g8 + 8 * ri));
-          acc[mt][2 * ri] = fmaf(acc[mt][2 * ri], al0, vcs * fmaf(sv, O[mt][2 * ri], zp0));
-          acc[mt][2 * ri + 1] = fmaf(acc[mt][2 * ri + 1], al1, vcs * fmaf(sv, O[mt][2 * ri + 1], zp1));
+          const float svr = ri ? sv1 : sv0;   // step with the codes' placement undone, per row half
+          acc[mt][2 * ri] = fmaf(acc[mt][2 * ri], al0, vcs * fmaf(svr, O[mt][2 * ri], zp0));
+          acc[mt][2 * ri + 1] = fmaf(acc[mt][2 * ri + 1], al1, vcs * fmaf(svr, O[mt][2 * ri + 1], zp1));
         }
     }
     __syncwarp();
