@@ -24,6 +24,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <atomic>
 #include <mutex>
 
@@ -45,7 +46,15 @@ struct QuantSmem {
   float zmin[4], zmax[4];
   alignas(16) uint8_t rec[kScaleRec];    // staged scale record
   alignas(8) uint64_t bar[2];
+  uint32_t tmem;                         // tensor-memory base of this CTA's R stash
 };
+
+// Tensor memory holds each tile's rotated R (fp32, 128 lanes x 128 columns =
+// 64 KB) from the rotation until quantisation, so R is computed once.  A CTA
+// allocates kTmemCols columns once; at most kMaxCtasPerSm CTAs share an SM's
+// 512 columns, so the allocation never waits.
+constexpr int kTmemCols = 128;
+constexpr int kMaxCtasPerSm = 512 / kTmemCols;
 
 // byte offset of (row t, 16-byte chunk c16 in 0..15) inside one stage
 __device__ __forceinline__ uint32_t xoff(int t, int c16) {
@@ -119,6 +128,48 @@ __device__ __forceinline__ uint32_t bfi(uint32_t x, uint32_t y, int pos, int len
   asm("bfi.b32 %0, %1, %2, %3, %4;\n" : "=r"(r) : "r"(x), "r"(y), "r"(pos), "r"(len));
   return r;
 }
+
+// ------------------------------------------------------------ tensor memory
+
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem) {   // whole warp
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_u32(dst_smem)),
+               "n"(kTmemCols) : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t base) {     // whole warp
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(base), "n"(kTmemCols) : "memory");
+}
+__device__ __forceinline__ void tmem_fence_before_sync() {
+  asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+}
+__device__ __forceinline__ void tmem_fence_after_sync() {
+  asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+}
+
+// 32 consecutive columns of this thread's lane <-> v[0..31]
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};\n" ::"r"(taddr),
+      "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]), "f"(v[8]), "f"(v[9]),
+      "f"(v[10]), "f"(v[11]), "f"(v[12]), "f"(v[13]), "f"(v[14]), "f"(v[15]), "f"(v[16]), "f"(v[17]), "f"(v[18]),
+      "f"(v[19]), "f"(v[20]), "f"(v[21]), "f"(v[22]), "f"(v[23]), "f"(v[24]), "f"(v[25]), "f"(v[26]), "f"(v[27]),
+      "f"(v[28]), "f"(v[29]), "f"(v[30]), "f"(v[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n"
+      : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]), "=f"(v[7]), "=f"(v[8]),
+        "=f"(v[9]), "=f"(v[10]), "=f"(v[11]), "=f"(v[12]), "=f"(v[13]), "=f"(v[14]), "=f"(v[15]), "=f"(v[16]),
+        "=f"(v[17]), "=f"(v[18]), "=f"(v[19]), "=f"(v[20]), "=f"(v[21]), "=f"(v[22]), "=f"(v[23]), "=f"(v[24]),
+        "=f"(v[25]), "=f"(v[26]), "=f"(v[27]), "=f"(v[28]), "=f"(v[29]), "=f"(v[30]), "=f"(v[31])
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
 
 // ---------------------------------------------------------------- rotation
 
@@ -218,6 +269,11 @@ __device__ __forceinline__ void quantize_tile(const QuantArgs& p, QuantSmem& sm,
   // ---- 2. rotate
   float A[128];
   if (SIDE == 0) rotate_k(xs, warp, lane, A); else rotate_v(xs, warp, lane, A);
+  // stash R in this warp's 32 TMEM lanes (lane field: bits 31..16, column: 15..0)
+  const uint32_t tr = sm.tmem + (static_cast<uint32_t>(32 * warp) << 16);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) tmem_st32(tr + 32 * q, A + 32 * q);
+  tmem_wait_st();
 #pragma unroll
   for (int i = 0; i < 128; i += 2) {
     const float2 s2 = __fmul2_rn(f2(A[i], A[i + 1]), f2(A[i], A[i + 1]));
@@ -366,9 +422,11 @@ __device__ __forceinline__ void quantize_tile(const QuantArgs& p, QuantSmem& sm,
   }
   __syncthreads();
 
-  // ---- 4. quantise: recompute R (same arithmetic), Z, zero/step, codes
+  // ---- 4. quantise: R back from tensor memory, Z, zero/step, codes
   float Z[128];
-  if (SIDE == 0) rotate_k(xs, warp, lane, Z); else rotate_v(xs, warp, lane, Z);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) tmem_ld32(tr + 32 * q, Z + 32 * q);
+  tmem_wait_ld();
   float zlo = 3.402823466e38f, zhi = -3.402823466e38f;
   if (SIDE == 0) {
     float mtv[4];
@@ -516,7 +574,10 @@ __global__ void __launch_bounds__(kQThreads, KVARN_Q_MIN_CTAS) quantize_kernel(c
     mbar_init(&sm.bar[1], 1);
     fence_barrier_init();
   }
+  if (tid < 32) tmem_alloc(&sm.tmem);
+  tmem_fence_before_sync();
   __syncthreads();
+  tmem_fence_after_sync();
   int64_t id = blockIdx.x;
   if (id < total && tid == 0) {
     int side, h;
@@ -543,7 +604,7 @@ __global__ void __launch_bounds__(kQThreads, KVARN_Q_MIN_CTAS) quantize_kernel(c
       // let the copies still in flight land before the shared memory is released
       (void)mbar_wait_bounded(&sm.bar[stage], (it >> 1) & 1);
       if (nxt < total) (void)mbar_wait_bounded(&sm.bar[stage ^ 1], ((it + 1) >> 1) & 1);
-      return;
+      break;
     }
     // which paged block: slot_mapping[128 * grp] must start a block of the pool
     const int64_t slot = p.slot_mapping[grp * kTile];
@@ -557,6 +618,11 @@ __global__ void __launch_bounds__(kQThreads, KVARN_Q_MIN_CTAS) quantize_kernel(c
     }
     __syncthreads();   // stage `stage` and the shared scratch are free again
   }
+  // every path reaches here with the CTA converged (the timeout break is CTA-uniform)
+  tmem_fence_before_sync();
+  __syncthreads();
+  tmem_fence_after_sync();
+  if (tid < 32) tmem_dealloc(sm.tmem);
 }
 
 // ---------------------------------------------------------------- host side
@@ -588,6 +654,30 @@ cudaError_t make_map(CUtensorMap* m, const __half* base, int hkv, int64_t num_to
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// CTAs of `fn` that fit on one SM by registers, shared memory and threads.  The
+// runtime's occupancy query answers 1 for any kernel that allocates tensor
+// memory, whatever its footprint, so the persistent grid is sized from the
+// kernel's own resources instead (the tensor-memory bound is applied by the caller).
+cudaError_t resident_ctas(const void* fn, int dyn_smem, int dev, int* out) {
+  cudaFuncAttributes fa;
+  cudaError_t e = cudaFuncGetAttributes(&fa, fn);
+  if (e != cudaSuccess) return e;
+  int regs_sm = 0, smem_sm = 0, thr_sm = 0, smem_rsv = 0, ctas_sm = 0;
+  if ((e = cudaDeviceGetAttribute(&regs_sm, cudaDevAttrMaxRegistersPerMultiprocessor, dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&thr_sm, cudaDevAttrMaxThreadsPerMultiProcessor, dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&smem_rsv, cudaDevAttrReservedSharedMemoryPerBlock, dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&ctas_sm, cudaDevAttrMaxBlocksPerMultiprocessor, dev)) != cudaSuccess) return e;
+  const int warps = (kQThreads + 31) / 32;
+  const int regs_warp = ((fa.numRegs * 32 + 255) / 256) * 256;   // allocated per warp in units of 256
+  int occ = ctas_sm;
+  occ = std::min(occ, regs_sm / std::max(1, regs_warp * warps));
+  occ = std::min(occ, smem_sm / std::max(1, static_cast<int>(fa.sharedSizeBytes) + dyn_smem + smem_rsv));
+  occ = std::min(occ, thr_sm / kQThreads);
+  *out = occ;
+  return cudaSuccess;
+}
+
 template <int KB, int VB>
 cudaError_t launch_q(const QuantArgs& p, cudaStream_t stream) {
   static std::atomic<uint64_t> configured{0};   // one bit per device ordinal
@@ -601,12 +691,14 @@ cudaError_t launch_q(const QuantArgs& p, cudaStream_t stream) {
   if ((configured.load(std::memory_order_acquire) & bit) == 0) {
     e = cudaFuncSetAttribute(quantize_kernel<KB, VB>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    int occ = 0, n = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, quantize_kernel<KB, VB>, kQThreads, smem);
-    if (e != cudaSuccess) return e;
+    int n = 0;
     e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
-    ctas_per_sm[dev & 63] = occ > 0 ? occ : 1;
+    int occ = 0;
+    e = resident_ctas(reinterpret_cast<const void*>(quantize_kernel<KB, VB>), smem, dev, &occ);
+    if (e != cudaSuccess) return e;
+    // each resident CTA holds kTmemCols of the SM's 512 tensor-memory columns
+    ctas_per_sm[dev & 63] = occ < 1 ? 1 : (occ > kMaxCtasPerSm ? kMaxCtasPerSm : occ);
     sms[dev & 63] = n;
     configured.fetch_or(bit, std::memory_order_acq_rel);
   }
