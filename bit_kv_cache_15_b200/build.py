@@ -16,7 +16,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libkvarn.so")
 SOURCES = ["kvarn_api.cu", "quantize.cu", "decode.cu", "baseline.cu"]
-HEADERS = ["common.cuh", "kvarn_internal.h"]
+HEADERS = ["common.cuh", "kvarn_internal.h", "quant_tile.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

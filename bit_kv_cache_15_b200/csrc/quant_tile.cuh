@@ -1,0 +1,541 @@
+// quant_tile.cuh -- one KVarN tile quantised by one 128-thread CTA (sm_100a).
+//
+// The four stages of [hypho] "KV-cache 量化终于能跑生产了？KVarN …", section
+// 它怎么做到的：四步流水线 (= [lehuy] "KVarN: Backend lượng tử hóa KV-cache …",
+// section Cơ chế hoạt động) after the tile is staged in shared memory:
+//   2 rotate  R = X H along channels.  H128 = H8 (x) H16 (Kronecker), so the
+//             16-channel factor runs on the tensor cores (mma.m16n8k16 against
+//             a +-1 fp16 H16) and the 8-group factor is an in-register
+//             butterfly across the eight mma results each lane holds;
+//   3 normalise  N passes of channel RMS then token RMS in base-2 log space:
+//             A = R*R stays in registers; each pass is packed f32x2 FMAs, a
+//             warp reduce-scatter and (for channels) a 4-warp shared sum;
+//   4 quantise   Z = (R * fp32(2^-Lt)) * fp32(2^-Lc) from the stored fp16
+//             log-scales, one zero/step per tile from min/max, codes =
+//             clamp(rne((Z - zero) * (1/step)));
+//   5 pack    codes in the decode's mma fragment order, 16-byte stores.
+// The K-side rotation uses X as the mma A operand and the V side as the B
+// operand, so after stage 2 each lane holds exactly the elements of the
+// decode kernel's mma fragments (K: rows tokens; V: rows channels): codes are
+// packed in registers and written with no cross-lane traffic.
+// Used by the quantise-on-write kernel and by the decode kernel's append path.
+#pragma once
+#include "common.cuh"
+#include "kvarn_internal.h"
+
+namespace kvarn {
+namespace qt {
+
+constexpr int kQThreads = 128;
+constexpr int kBox = 128 * 128;       // one 64-channel box: 128 rows of 128 bytes
+
+// Per-CTA scratch of one tile's normalisation and quantisation.
+struct QuantScratch {
+  float red[4][kHeadDim];                // per-warp channel partial sums
+  float u[kHeadDim];                     // channel weights 2^(-2 lc)
+  float mt[kTile];                       // fp32(2^-Lt)
+  float mc[kHeadDim];                    // fp32(2^-Lc)
+  float zmin[4], zmax[4];
+  alignas(16) uint8_t rec[kScaleRec];    // staged scale record
+};
+
+// Tensor memory can hold a tile's rotated R (fp32, 128 lanes x 128 columns =
+// 64 KB) from the rotation until quantisation, so R is computed once.
+constexpr int kTmemCols = 128;
+
+// byte offset of (row t, 16-byte chunk c16 in 0..15) inside one stage
+__device__ __forceinline__ uint32_t xoff(int t, int c16) {
+  return (c16 >> 3) * kBox + t * 128 + (((c16 & 7) ^ (t & 7)) << 4);
+}
+
+__device__ __forceinline__ float lg2_approx(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// 1/2 log2 of the mean square (sum / 128), floored at 2^-48
+__device__ __forceinline__ float log2_scale(float sum_sq) {
+  return 0.5f * (lg2_approx(fmaxf(sum_sq, 4.547473508864641e-13f)) - 7.0f);   // 2^-41
+}
+
+// fp16 bit pattern of the Hadamard sign H16[r][c] = (-1)^popcount(r & c).
+__device__ __forceinline__ uint32_t h16_bits(int r, int c) {
+  return (__popc(r & c) & 1) ? 0xBC00u : 0x3C00u;
+}
+__device__ __forceinline__ uint32_t h16_pair(int r0, int c0, int r1, int c1) {
+  return h16_bits(r0, c0) | (h16_bits(r1, c1) << 16);
+}
+
+// In-register 8-point Walsh-Hadamard transforms (Sylvester order) of two
+// independent vectors at once: lane .x of v is one vector, lane .y the other.
+__device__ __forceinline__ void fwht8x2(float2 (&v)[8]) {
+#pragma unroll
+  for (int hl = 1; hl < 8; hl <<= 1) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if ((i & hl) == 0) {
+        const float2 a = v[i], b = v[i + hl];
+        v[i] = __fadd2_rn(a, b);
+        v[i + hl] = __fadd2_rn(a, make_float2(-b.x, -b.y));
+      }
+    }
+  }
+}
+
+// One reduce-scatter step across lanes (lane ^ mask): the first N/2 entries
+// of v end up holding the half this lane keeps, summed with its partner's.
+template <int N>
+__device__ __forceinline__ void rs_step(float* v, int mask, int lane) {
+  const bool up = (lane & mask) != 0;
+#pragma unroll
+  for (int i = 0; i < N / 2; ++i) {
+    const float send = up ? v[i] : v[i + N / 2];
+    const float keep = up ? v[i + N / 2] : v[i];
+    v[i] = keep + __shfl_xor_sync(0xffffffffu, send, mask);
+  }
+}
+
+__device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
+
+__device__ __forceinline__ float min3(float a, float b, float c) {
+  float r;
+  asm("min.f32 %0, %1, %2, %3;\n" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;\n" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// insert the low `len` bits of x into y at bit `pos`
+__device__ __forceinline__ uint32_t bfi(uint32_t x, uint32_t y, int pos, int len) {
+  uint32_t r;
+  asm("bfi.b32 %0, %1, %2, %3, %4;\n" : "=r"(r) : "r"(x), "r"(y), "r"(pos), "r"(len));
+  return r;
+}
+
+// ------------------------------------------------------------ tensor memory
+
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem) {   // whole warp
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_u32(dst_smem)),
+               "n"(kTmemCols) : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t base) {     // whole warp
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(base), "n"(kTmemCols) : "memory");
+}
+__device__ __forceinline__ void tmem_fence_before_sync() {
+  asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+}
+__device__ __forceinline__ void tmem_fence_after_sync() {
+  asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+}
+
+// 32 consecutive columns of this thread's lane <-> v[0..31]
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};\n" ::"r"(taddr),
+      "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]), "f"(v[8]), "f"(v[9]),
+      "f"(v[10]), "f"(v[11]), "f"(v[12]), "f"(v[13]), "f"(v[14]), "f"(v[15]), "f"(v[16]), "f"(v[17]), "f"(v[18]),
+      "f"(v[19]), "f"(v[20]), "f"(v[21]), "f"(v[22]), "f"(v[23]), "f"(v[24]), "f"(v[25]), "f"(v[26]), "f"(v[27]),
+      "f"(v[28]), "f"(v[29]), "f"(v[30]), "f"(v[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n"
+      : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]), "=f"(v[7]), "=f"(v[8]),
+        "=f"(v[9]), "=f"(v[10]), "=f"(v[11]), "=f"(v[12]), "=f"(v[13]), "=f"(v[14]), "=f"(v[15]), "=f"(v[16]),
+        "=f"(v[17]), "=f"(v[18]), "=f"(v[19]), "=f"(v[20]), "=f"(v[21]), "=f"(v[22]), "=f"(v[23]), "=f"(v[24]),
+        "=f"(v[25]), "=f"(v[26]), "=f"(v[27]), "=f"(v[28]), "=f"(v[29]), "=f"(v[30]), "=f"(v[31])
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
+
+// ---------------------------------------------------------------- rotation
+
+// K side: thread holds R at t = 16*(2w+ml) + g + 8*ri, d = 16*a + 8*nb + 2*c + rj
+// in R[((ml*8 + a)*2 + nb)*4 + 2*ri + rj]   (g = lane/4, c = lane%4).
+__device__ __forceinline__ void rotate_k(uint32_t xs, int warp, int lane, float (&R)[128]) {
+  const int g = lane >> 2, c = lane & 3;
+  uint32_t hb0[2], hb1[2];
+#pragma unroll
+  for (int nb = 0; nb < 2; ++nb) {
+    const int n = 8 * nb + g;
+    hb0[nb] = h16_pair(2 * c, n, 2 * c + 1, n);
+    hb1[nb] = h16_pair(2 * c + 8, n, 2 * c + 9, n);
+  }
+  const int mi = lane >> 3;
+#pragma unroll
+  for (int ml = 0; ml < 2; ++ml) {
+    const int row = 16 * (2 * warp + ml) + (lane & 7) + 8 * (mi & 1);
+    float C[8][2][4];
+#pragma unroll
+    for (int a = 0; a < 8; ++a) {
+      uint32_t a0, a1, a2, a3;
+      ldmatrix_x4(xs + xoff(row, 2 * a + (mi >> 1)), a0, a1, a2, a3);
+#pragma unroll
+      for (int nb = 0; nb < 2; ++nb) {
+#pragma unroll
+        for (int r = 0; r < 4; ++r) C[a][nb][r] = 0.f;
+        mma_f16(C[a][nb], a0, a1, a2, a3, hb0[nb], hb1[nb]);
+      }
+    }
+#pragma unroll
+    for (int nb = 0; nb < 2; ++nb) {
+#pragma unroll
+      for (int r = 0; r < 4; r += 2) {
+        float2 v[8];
+#pragma unroll
+        for (int a = 0; a < 8; ++a) v[a] = make_float2(C[a][nb][r], C[a][nb][r + 1]);
+        fwht8x2(v);
+#pragma unroll
+        for (int a = 0; a < 8; ++a) {
+          R[((ml * 8 + a) * 2 + nb) * 4 + r] = v[a].x;
+          R[((ml * 8 + a) * 2 + nb) * 4 + r + 1] = v[a].y;
+        }
+      }
+    }
+  }
+}
+
+// V side: thread holds R at t = 8*(4w+ntl) + 2*c + rj, d = 16*a + g + 8*ri
+// in R[(ntl*8 + a)*4 + 2*ri + rj].
+__device__ __forceinline__ void rotate_v(uint32_t xs, int warp, int lane, float (&R)[128]) {
+  const int g = lane >> 2, c = lane & 3;
+  const uint32_t ha0 = h16_pair(g, 2 * c, g, 2 * c + 1);
+  const uint32_t ha1 = h16_pair(g + 8, 2 * c, g + 8, 2 * c + 1);
+  const uint32_t ha2 = h16_pair(g, 2 * c + 8, g, 2 * c + 9);
+  const uint32_t ha3 = h16_pair(g + 8, 2 * c + 8, g + 8, 2 * c + 9);
+  const int mi = lane >> 3;
+#pragma unroll
+  for (int ntl = 0; ntl < 4; ++ntl) {
+    const int row = 8 * (4 * warp + ntl) + (lane & 7);
+    float C[8][4];
+#pragma unroll
+    for (int ap = 0; ap < 4; ++ap) {
+      uint32_t r0, r1, r2, r3;
+      ldmatrix_x4(xs + xoff(row, 4 * ap + mi), r0, r1, r2, r3);
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        C[2 * ap][r] = 0.f;
+        C[2 * ap + 1][r] = 0.f;
+      }
+      mma_f16(C[2 * ap], ha0, ha1, ha2, ha3, r0, r1);
+      mma_f16(C[2 * ap + 1], ha0, ha1, ha2, ha3, r2, r3);
+    }
+#pragma unroll
+    for (int r = 0; r < 4; r += 2) {
+      float2 v[8];
+#pragma unroll
+      for (int a = 0; a < 8; ++a) v[a] = make_float2(C[a][r], C[a][r + 1]);
+      fwht8x2(v);
+#pragma unroll
+      for (int a = 0; a < 8; ++a) {
+        R[(ntl * 8 + a) * 4 + r] = v[a].x;
+        R[(ntl * 8 + a) * 4 + r + 1] = v[a].y;
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------- the tile
+
+// Where one tile's results go.
+struct TileOut {
+  uint8_t* codes;        // this side's code block (2048 * BITS bytes, 16-byte aligned)
+  uint8_t* scales;       // this side's 528-byte scale record
+  float* dbg;            // nullable: fp32 log-scales before rounding (256 floats)
+  int iters;
+};
+
+// Stages 2-5 for the fp16 tile staged at shared address xs (xoff layout), by
+// all 128 threads of the CTA.  STASH: keep R in tensor memory at tmem (this
+// CTA's allocation) between the rotation and quantisation; otherwise the
+// rotation is run a second time from the staged tile (same arithmetic).
+template <int SIDE, int BITS, bool STASH>
+__device__ __forceinline__ void quantize_tile(const TileOut& o, QuantScratch& sm, uint32_t xs, uint32_t tmem) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, c = lane & 3;
+
+  // ---- 2. rotate
+  float A[128];
+  if (SIDE == 0) rotate_k(xs, warp, lane, A); else rotate_v(xs, warp, lane, A);
+  // stash R in this warp's 32 TMEM lanes (lane field: bits 31..16, column: 15..0)
+  const uint32_t tr = tmem + (static_cast<uint32_t>(32 * warp) << 16);
+  if (STASH) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) tmem_st32(tr + 32 * q, A + 32 * q);
+    tmem_wait_st();
+  }
+#pragma unroll
+  for (int i = 0; i < 128; i += 2) {
+    const float2 s2 = __fmul2_rn(f2(A[i], A[i + 1]), f2(A[i], A[i + 1]));
+    A[i] = s2.x;
+    A[i + 1] = s2.y;
+  }
+
+  // ---- 3. normalise
+  constexpr int NT = SIDE == 0 ? 4 : 8;   // tokens per thread
+  float wt[NT];                           // token weights 2^(-2 lt)
+#pragma unroll
+  for (int i = 0; i < NT; ++i) wt[i] = 1.f;
+  float lt_own = 0.f, lc_own = 0.f;
+
+  for (int it = 0; it < o.iters; ++it) {
+    // channel pass: partial sums over this thread's tokens
+    if (SIDE == 0) {
+      float s[32];   // index a*4 + nb*2 + rj
+#pragma unroll
+      for (int a = 0; a < 8; ++a)
+#pragma unroll
+        for (int nb = 0; nb < 2; ++nb) {
+          float2 acc = f2(0.f, 0.f);
+#pragma unroll
+          for (int ml = 0; ml < 2; ++ml)
+#pragma unroll
+            for (int ri = 0; ri < 2; ++ri) {
+              const int i = ((ml * 8 + a) * 2 + nb) * 4 + 2 * ri;
+              const float w = wt[ml * 2 + ri];
+              acc = __ffma2_rn(f2(A[i], A[i + 1]), f2(w, w), acc);
+            }
+          s[a * 4 + nb * 2] = acc.x;
+          s[a * 4 + nb * 2 + 1] = acc.y;
+        }
+      rs_step<32>(s, 16, lane);
+      rs_step<16>(s, 8, lane);
+      rs_step<8>(s, 4, lane);
+      *reinterpret_cast<float2*>(&sm.red[warp][16 * g + 2 * c]) = f2(s[0], s[1]);
+      *reinterpret_cast<float2*>(&sm.red[warp][16 * g + 8 + 2 * c]) = f2(s[2], s[3]);
+    } else {
+      float s[16];   // index a*2 + ri
+#pragma unroll
+      for (int a = 0; a < 8; ++a)
+#pragma unroll
+        for (int ri = 0; ri < 2; ++ri) {
+          float2 acc = f2(0.f, 0.f);
+#pragma unroll
+          for (int ntl = 0; ntl < 4; ++ntl) {
+            const int i = (ntl * 8 + a) * 4 + 2 * ri;
+            acc = __ffma2_rn(f2(A[i], A[i + 1]), f2(wt[ntl * 2], wt[ntl * 2 + 1]), acc);
+          }
+          s[a * 2 + ri] = acc.x + acc.y;
+        }
+      rs_step<16>(s, 2, lane);
+      rs_step<8>(s, 1, lane);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int a = 2 * c + (k >> 1), ri = k & 1;
+        sm.red[warp][16 * a + g + 8 * ri] = s[k];
+      }
+    }
+    __syncthreads();
+    {
+      const float tot = (sm.red[0][tid] + sm.red[1][tid]) + (sm.red[2][tid] + sm.red[3][tid]);
+      lc_own = log2_scale(tot);
+      sm.u[tid] = ex2_fast(-2.f * lc_own);
+    }
+    __syncthreads();
+
+    // token pass
+    if (SIDE == 0) {
+      float2 uu[16];   // (a, nb) -> channels 16a + 8nb + 2c + {0,1}
+#pragma unroll
+      for (int a = 0; a < 8; ++a)
+#pragma unroll
+        for (int nb = 0; nb < 2; ++nb)
+          uu[a * 2 + nb] = *reinterpret_cast<const float2*>(&sm.u[16 * a + 8 * nb + 2 * c]);
+      float s[4];    // index ml*2 + ri
+#pragma unroll
+      for (int ml = 0; ml < 2; ++ml)
+#pragma unroll
+        for (int ri = 0; ri < 2; ++ri) {
+          float2 acc[4] = {f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f)};   // 4 chains for ILP
+#pragma unroll
+          for (int a = 0; a < 8; ++a)
+#pragma unroll
+            for (int nb = 0; nb < 2; ++nb) {
+              const int i = ((ml * 8 + a) * 2 + nb) * 4 + 2 * ri;
+              acc[(a & 1) * 2 + nb] = __ffma2_rn(f2(A[i], A[i + 1]), uu[a * 2 + nb], acc[(a & 1) * 2 + nb]);
+            }
+          const float2 t01 = __fadd2_rn(acc[0], acc[1]), t23 = __fadd2_rn(acc[2], acc[3]);
+          const float2 t = __fadd2_rn(t01, t23);
+          s[ml * 2 + ri] = t.x + t.y;
+        }
+      rs_step<4>(s, 2, lane);
+      rs_step<2>(s, 1, lane);
+      lt_own = log2_scale(s[0]);
+      const float wown = ex2_fast(-2.f * lt_own);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) wt[k] = __shfl_sync(0xffffffffu, wown, (lane & ~3) | k);
+    } else {
+      float uu[16];
+#pragma unroll
+      for (int a = 0; a < 8; ++a)
+#pragma unroll
+        for (int ri = 0; ri < 2; ++ri) uu[a * 2 + ri] = sm.u[16 * a + g + 8 * ri];
+      float s[8];    // index ntl*2 + rj
+#pragma unroll
+      for (int ntl = 0; ntl < 4; ++ntl) {
+        float2 acc[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};   // 2 chains for ILP
+#pragma unroll
+        for (int a = 0; a < 8; ++a)
+#pragma unroll
+          for (int ri = 0; ri < 2; ++ri) {
+            const int i = (ntl * 8 + a) * 4 + 2 * ri;
+            const float uv = uu[a * 2 + ri];
+            acc[ri] = __ffma2_rn(f2(A[i], A[i + 1]), f2(uv, uv), acc[ri]);
+          }
+        const float2 t = __fadd2_rn(acc[0], acc[1]);
+        s[ntl * 2] = t.x;
+        s[ntl * 2 + 1] = t.y;
+      }
+      rs_step<8>(s, 16, lane);
+      rs_step<4>(s, 8, lane);
+      rs_step<2>(s, 4, lane);
+      lt_own = log2_scale(s[0]);
+      const float wown = ex2_fast(-2.f * lt_own);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) wt[k] = __shfl_sync(0xffffffffu, wown, c | (k << 2));
+    }
+  }
+
+  // ---- stored fp16 log-scales and their fp32 multipliers
+  const int t_own = (SIDE == 0) ? 16 * (2 * warp + ((lane >> 1) & 1)) + g + 8 * (lane & 1)
+                                : 8 * (4 * warp + (lane >> 3)) + 2 * c + ((lane >> 2) & 1);
+  const __half Lt16 = __float2half_rn(lt_own);
+  const __half Lc16 = __float2half_rn(lc_own);
+  sm.mt[t_own] = __double2float_rn(exp2(-static_cast<double>(__half2float(Lt16))));
+  sm.mc[tid] = __double2float_rn(exp2(-static_cast<double>(__half2float(Lc16))));
+  reinterpret_cast<__half*>(sm.rec)[t_own] = Lt16;
+  reinterpret_cast<__half*>(sm.rec + 256)[tid] = Lc16;
+  if (o.dbg != nullptr) {
+    o.dbg[t_own] = lt_own;
+    o.dbg[128 + tid] = lc_own;
+  }
+  __syncthreads();
+
+  // ---- 4. quantise: R again (from tensor memory, or recomputed), Z, zero/step, codes
+  float Z[128];
+  if (STASH) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) tmem_ld32(tr + 32 * q, Z + 32 * q);
+    tmem_wait_ld();
+  } else {
+    if (SIDE == 0) rotate_k(xs, warp, lane, Z); else rotate_v(xs, warp, lane, Z);
+  }
+  float zlo = 3.402823466e38f, zhi = -3.402823466e38f;
+  if (SIDE == 0) {
+    float mtv[4];
+#pragma unroll
+    for (int ml = 0; ml < 2; ++ml)
+#pragma unroll
+      for (int ri = 0; ri < 2; ++ri) mtv[ml * 2 + ri] = sm.mt[16 * (2 * warp + ml) + g + 8 * ri];
+#pragma unroll
+    for (int a = 0; a < 8; ++a)
+#pragma unroll
+      for (int nb = 0; nb < 2; ++nb) {
+        const float2 mc2 = *reinterpret_cast<const float2*>(&sm.mc[16 * a + 8 * nb + 2 * c]);
+#pragma unroll
+        for (int ml = 0; ml < 2; ++ml)
+#pragma unroll
+          for (int ri = 0; ri < 2; ++ri) {
+            const int i = ((ml * 8 + a) * 2 + nb) * 4 + 2 * ri;
+            const float m = mtv[ml * 2 + ri];
+            const float2 z = __fmul2_rn(__fmul2_rn(f2(Z[i], Z[i + 1]), f2(m, m)), mc2);
+            Z[i] = z.x;
+            Z[i + 1] = z.y;
+            zlo = min3(zlo, z.x, z.y);
+            zhi = max3(zhi, z.x, z.y);
+          }
+      }
+  } else {
+    float2 mtv[4];
+#pragma unroll
+    for (int ntl = 0; ntl < 4; ++ntl) mtv[ntl] = *reinterpret_cast<const float2*>(&sm.mt[8 * (4 * warp + ntl) + 2 * c]);
+#pragma unroll
+    for (int a = 0; a < 8; ++a)
+#pragma unroll
+      for (int ri = 0; ri < 2; ++ri) {
+        const float mcv = sm.mc[16 * a + g + 8 * ri];
+#pragma unroll
+        for (int ntl = 0; ntl < 4; ++ntl) {
+          const int i = (ntl * 8 + a) * 4 + 2 * ri;
+          const float2 z = __fmul2_rn(__fmul2_rn(f2(Z[i], Z[i + 1]), mtv[ntl]), f2(mcv, mcv));
+          Z[i] = z.x;
+          Z[i + 1] = z.y;
+          zlo = min3(zlo, z.x, z.y);
+          zhi = max3(zhi, z.x, z.y);
+        }
+      }
+  }
+  const float zl = warp_min(zlo);
+  const float zh = warp_max(zhi);
+  if (lane == 0) {
+    sm.zmin[warp] = zl;
+    sm.zmax[warp] = zh;
+  }
+  __syncthreads();
+  const float zero = fminf(fminf(sm.zmin[0], sm.zmin[1]), fminf(sm.zmin[2], sm.zmin[3]));
+  const float zmx = fmaxf(fmaxf(sm.zmax[0], sm.zmax[1]), fmaxf(sm.zmax[2], sm.zmax[3]));
+  constexpr int LB = (1 << BITS) - 1;
+  float step = __fdiv_rn(__fsub_rn(zmx, zero), static_cast<float>(LB));
+  if (step == 0.f) step = 1.f;
+  const float inv = __fdiv_rn(1.f, step);
+
+  // codes: y = (Z - zero) * inv >= 0, rounded to nearest even by adding 1.5 * 2^23
+  // (exact for y < 2^22); packed in the fragment order (block bl, register j, half h)
+  constexpr int PER = 16 / BITS;          // register pairs per 32-bit word
+  constexpr int NW = 64 / PER;            // words per thread (= 4*BITS)
+  constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23
+  uint32_t words[NW];
+#pragma unroll
+  for (int i = 0; i < NW; ++i) words[i] = 0u;
+#pragma unroll
+  for (int bl = 0; bl < 16; ++bl)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      int idx;                             // index of the (h = 0) element; h = 1 is idx + 1
+      if (SIDE == 0) {   // bl = ml*8 + a;  j = ri + 2*nb;  h = rj
+        const int ml = bl >> 3, a = bl & 7, nb = j >> 1, ri = j & 1;
+        idx = ((ml * 8 + a) * 2 + nb) * 4 + 2 * ri;
+      } else {           // bl = (ntl>>1)*8 + a;  j = ri + 2*(ntl&1);  h = rj
+        const int ntl = 2 * (bl >> 3) + (j >> 1), a = bl & 7, ri = j & 1;
+        idx = (ntl * 8 + a) * 4 + 2 * ri;
+      }
+      const float2 y = __fmul2_rn(__fadd2_rn(f2(Z[idx], Z[idx + 1]), f2(-zero, -zero)), f2(inv, inv));
+      const float2 r = __fadd2_rn(y, f2(kMagic, kMagic));
+      // 0 <= y <= 2^b - 1 up to rounding, so rne(y) sits in the low BITS bits of r
+      const int rho = 4 * bl + j;
+      words[rho / PER] = bfi(__float_as_uint(r.x), words[rho / PER], BITS * (rho % PER), BITS);
+      words[rho / PER] = bfi(__float_as_uint(r.y), words[rho / PER], BITS * (rho % PER) + 16, BITS);
+    }
+
+  // ---- 5. store codes (16-byte chunks, lane-interleaved) and the scale record
+  uint8_t* dst = o.codes;
+#pragma unroll
+  for (int cc = 0; cc < BITS; ++cc) {
+    const uint4 v4 = make_uint4(words[4 * cc], words[4 * cc + 1], words[4 * cc + 2], words[4 * cc + 3]);
+    *reinterpret_cast<uint4*>(dst + ((warp * BITS + cc) * 32 + lane) * 16) = v4;
+  }
+  if (tid == 0) {
+    float* tailp = reinterpret_cast<float*>(sm.rec + 512);
+    tailp[0] = zero;
+    tailp[1] = step;
+    tailp[2] = 0.f;
+    tailp[3] = 0.f;
+  }
+  __syncthreads();
+  if (tid < kScaleRec / 16) {
+    *reinterpret_cast<uint4*>(o.scales + tid * 16) = *reinterpret_cast<const uint4*>(sm.rec + tid * 16);
+  }
+}
+
+}  // namespace qt
+}  // namespace kvarn
