@@ -29,6 +29,7 @@
 
 #include "common.cuh"
 #include "kvarn_internal.h"
+#include "quant_tile.cuh"
 
 namespace kvarn {
 namespace {
@@ -68,6 +69,8 @@ struct DecodeTraits {
   static_assert(kStage % 16 == 0, "stage must stay 16-byte aligned");
   static_assert(kSmem <= 227 * 1024, "shared memory");
   static_assert(kDWarps * kDStages * 8 <= 128, "barrier area");
+  // the append path stages a 32 KB fp16 tile and the quantiser scratch below the barriers
+  static_assert(kBarOff >= 2 * qt::kBox + static_cast<int>(sizeof(qt::QuantScratch)), "append staging");
 };
 
 // Where a code of `slot` sits in its fp16 half-word for the mma: bit
@@ -106,9 +109,49 @@ __device__ __forceinline__ float hf(const __half* p, int i) { return __half2floa
 
 // ------------------------------------------------------------------ tail CTA
 
+// Quantise the full fp16 tail tile of (b, h) -- rows 0..126 from the tail
+// buffer, row 127 = the appended token -- into block block_table[b][L / 128]
+// (K then V), by the whole CTA, with the rotation recomputed (no tensor memory).
+template <int KB, int VB>
+__device__ void quantize_full_tail(const DecodeArgs& p, uint8_t* smem, int b, int h, int L) {
+  using namespace qt;
+  const int tid = threadIdx.x;
+  const int32_t blk = p.block_table[(int64_t)b * p.max_blocks + (L >> 7)];
+  if (blk < 0 || blk >= p.num_blocks) {
+    if (tid == 0) report_status(p.status, KVARN_DEV_BAD_BLOCK);
+    return;
+  }
+  QuantScratch& sq = *reinterpret_cast<QuantScratch*>(smem + 2 * kBox);
+  const uint32_t xs = smem_u32(smem);
+#pragma unroll 1
+  for (int side = 0; side < 2; ++side) {
+    const __half* src = p.tail + (((int64_t)b * 2 + side) * p.Hkv + h) * (int64_t)(kTile * kHeadDim);
+    const __half* nrow = (side == 0 ? p.k_new : p.v_new) + ((int64_t)b * p.Hkv + h) * kHeadDim;
+    // stage row t = tid into the swizzled layout the rotation reads
+    const uint4* row = reinterpret_cast<const uint4*>(tid == kTile - 1 ? nrow : src + (int64_t)tid * kHeadDim);
+#pragma unroll 4
+    for (int c16 = 0; c16 < 16; ++c16) {
+      const uint4 v = __ldg(row + c16);
+      *reinterpret_cast<uint4*>(smem + xoff(tid, c16)) = v;
+    }
+    __syncthreads();
+    TileOut o;
+    o.codes = p.packed_w + ((int64_t)blk * p.Hkv + h) * (int64_t)(2048 * (KB + VB)) + (side == 0 ? 0 : 2048 * KB);
+    o.scales = p.scales_w + (((int64_t)blk * p.Hkv + h) * 2 + side) * (int64_t)kScaleRec;
+    o.dbg = nullptr;
+    o.iters = p.iters;
+    if (side == 0) quantize_tile<0, KB, false>(o, sq, xs, 0u);
+    else quantize_tile<1, VB, false>(o, sq, xs, 0u);
+    __syncthreads();   // the staged tile and the scratch are free again
+  }
+}
+
+template <int KB, int VB>
 __device__ void decode_tail(const DecodeArgs& p, uint8_t* smem, float* qs, int b, int h, int L) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int tl = L & 127;
+  // with append, the step's own token (position L) is the tail's last row and
+  // is read from k_new / v_new; it is also written to the tail buffer
+  const int tl = (L & 127) + p.append;
   if (tl == 0) return;
   const int G = p.G;
   float* sc = reinterpret_cast<float*>(smem);  // [kMaxG][128] scores, then weights
@@ -118,13 +161,16 @@ __device__ void decode_tail(const DecodeArgs& p, uint8_t* smem, float* qs, int b
   const float sl = p.sm_scale * kLog2e;
   const __half* kt = p.tail + (((int64_t)b * 2 + 0) * p.Hkv + h) * (int64_t)(kTile * kHeadDim);
   const __half* vt = p.tail + (((int64_t)b * 2 + 1) * p.Hkv + h) * (int64_t)(kTile * kHeadDim);
+  // row tl - 1: the appended token, or the tail buffer's own row (never a null pointer)
+  const __half* klast = p.append ? p.k_new + ((int64_t)b * p.Hkv + h) * kHeadDim : kt + (int64_t)(tl - 1) * kHeadDim;
+  const __half* vlast = p.append ? p.v_new + ((int64_t)b * p.Hkv + h) * kHeadDim : vt + (int64_t)(tl - 1) * kHeadDim;
   {
     const int t = tid;
     float dots[kMaxG];
 #pragma unroll
     for (int g = 0; g < kMaxG; ++g) dots[g] = 0.f;
     if (t < tl) {
-      const uint4* row = reinterpret_cast<const uint4*>(kt + (int64_t)t * kHeadDim);
+      const uint4* row = reinterpret_cast<const uint4*>(t == tl - 1 ? klast : kt + (int64_t)t * kHeadDim);
 #pragma unroll 4
       for (int c8 = 0; c8 < 16; ++c8) {
         const uint4 raw = __ldg(row + c8);
@@ -172,7 +218,8 @@ __device__ void decode_tail(const DecodeArgs& p, uint8_t* smem, float* qs, int b
 #pragma unroll
   for (int g = 0; g < kMaxG; ++g) acc[g] = 0.f;
   for (int t = 0; t < tl; ++t) {
-    const float vv = __half2float(vt[(int64_t)t * kHeadDim + d]);
+    const __half* vrow = t == tl - 1 ? vlast : vt + (int64_t)t * kHeadDim;
+    const float vv = __half2float(vrow[d]);
 #pragma unroll
     for (int g = 0; g < kMaxG; ++g) acc[g] = fmaf(sc[g * 128 + t], vv, acc[g]);
   }
@@ -185,6 +232,17 @@ __device__ void decode_tail(const DecodeArgs& p, uint8_t* smem, float* qs, int b
       rec[3] = 0.f;
     }
     rec[4 + d] = acc[g];
+  }
+  if (p.append) {
+    const int r = L & 127;
+    __half* kw = p.tail_w + (((int64_t)b * 2 + 0) * p.Hkv + h) * (int64_t)(kTile * kHeadDim) + (int64_t)r * kHeadDim;
+    __half* vw = p.tail_w + (((int64_t)b * 2 + 1) * p.Hkv + h) * (int64_t)(kTile * kHeadDim) + (int64_t)r * kHeadDim;
+    kw[d] = klast[d];
+    vw[d] = vlast[d];
+    if (tl == kTile) {
+      __syncthreads();   // the scores area is reused for the staged tile
+      quantize_full_tail<KB, VB>(p, smem, b, h, L);
+    }
   }
 }
 
@@ -620,13 +678,13 @@ __device__ void combine_pair(const DecodeArgs& p, int b, int h, int L, bool vali
   for (int g = warp; g < p.G; g += kDWarps) {
     const int j = h * p.G + g;
     __half* o = p.out + ((int64_t)b * p.Hq + j) * kHeadDim + 4 * lane;
-    if (!valid || L == 0) {
+    if (!valid || L + p.append == 0) {
       *reinterpret_cast<uint2*>(o) = make_uint2(0u, 0u);
       continue;
     }
     const int n_full = L >> 7;
     const int nsv = (n_full + p.tiles_per_split - 1) / p.tiles_per_split;
-    const bool has_tail = (L & 127) != 0;
+    const bool has_tail = (L & 127) + p.append != 0;
     const float* rec = p.ws + ((int64_t)b * p.Hq + j) * (p.num_splits + 1) * kPartialFloats;
     const float* trec = rec + (int64_t)p.num_splits * kPartialFloats;
     float M = has_tail ? __ldcg(trec) : -INFINITY;
@@ -682,12 +740,12 @@ __global__ void __launch_bounds__(kDThreads, KVARN_D_MIN_CTAS) decode_kernel(con
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ int last_arrival;
   const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int L = p.seq_lens[b];
-  const bool valid = L >= 0 && L <= kTile * p.max_blocks;
+  const int L = p.seq_lens[b];   // before the step's own token when appending
+  const bool valid = L >= 0 && L + p.append <= kTile * p.max_blocks;
   if (!valid) {
     if (threadIdx.x == 0 && s == 0) report_status(p.status, KVARN_DEV_BAD_SEQ_LEN);
   } else if (s == p.num_splits) {
-    decode_tail(p, smem, reinterpret_cast<float*>(smem + DecodeTraits<KB, VB>::kQrotOff), b, h, L);
+    decode_tail<KB, VB>(p, smem, reinterpret_cast<float*>(smem + DecodeTraits<KB, VB>::kQrotOff), b, h, L);
   } else {
     decode_split<KB, VB>(p, smem, b, h, s, L);
   }

@@ -144,10 +144,11 @@ kvarn_status kvarn_quantize_tiles_debug(const void* k, const void* v, const int6
                        debug_logscales, dev_status, stream);
 }
 
-kvarn_status kvarn_decode_attention(const void* q, const void* packed_cache, const void* scales,
-                                    const void* fp16_tail, const int32_t* block_table, const int32_t* seq_lens,
-                                    void* out, const kvarn_decode_dims* dims, const kvarn_config* cfg,
-                                    void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream) {
+static kvarn_status decode_impl(const void* q, const void* k_new, const void* v_new, const void* packed_cache,
+                                const void* scales, const void* fp16_tail, const int32_t* block_table,
+                                const int32_t* seq_lens, void* out, const kvarn_decode_dims* dims,
+                                const kvarn_config* cfg, void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                                void* stream, int append) {
   kvarn_status st = kvarn_config_validate(cfg);
   if (st != KVARN_OK) return st;
   st = check_dims(dims, 8);
@@ -158,6 +159,8 @@ kvarn_status kvarn_decode_attention(const void* q, const void* packed_cache, con
     return KVARN_ERR_INVALID_ARGUMENT;
   if (!aligned16(q) || !aligned16(packed_cache) || !aligned16(scales) || !aligned16(fp16_tail) ||
       !aligned16(workspace) || (reinterpret_cast<uintptr_t>(out) & 7u) != 0)
+    return KVARN_ERR_INVALID_ARGUMENT;
+  if (append && (k_new == nullptr || v_new == nullptr || !aligned16(k_new) || !aligned16(v_new)))
     return KVARN_ERR_INVALID_ARGUMENT;
   const size_t need = workspace_for(dims->num_seqs, dims->num_q_heads, dims->num_kv_heads, dims->max_blocks_per_seq);
   if (workspace_bytes < need) return KVARN_ERR_WORKSPACE_TOO_SMALL;
@@ -184,7 +187,31 @@ kvarn_status kvarn_decode_attention(const void* q, const void* packed_cache, con
   kvarn::decode_geometry(p.B, p.Hkv, p.max_blocks, &p.tiles_per_split, &p.num_splits);
   p.sm_scale = effective_sm_scale(cfg);
   p.status = dev_status;
+  p.append = append;
+  p.k_new = static_cast<const __half*>(k_new);
+  p.v_new = static_cast<const __half*>(v_new);
+  p.tail_w = append ? static_cast<__half*>(const_cast<void*>(fp16_tail)) : nullptr;
+  p.packed_w = append ? static_cast<uint8_t*>(const_cast<void*>(packed_cache)) : nullptr;
+  p.scales_w = append ? static_cast<uint8_t*>(const_cast<void*>(scales)) : nullptr;
+  p.iters = cfg->sinkhorn_iters;
   return from_cuda(kvarn::launch_decode(p, static_cast<cudaStream_t>(stream)));
+}
+
+kvarn_status kvarn_decode_attention(const void* q, const void* packed_cache, const void* scales,
+                                    const void* fp16_tail, const int32_t* block_table, const int32_t* seq_lens,
+                                    void* out, const kvarn_decode_dims* dims, const kvarn_config* cfg,
+                                    void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream) {
+  return decode_impl(q, nullptr, nullptr, packed_cache, scales, fp16_tail, block_table, seq_lens, out, dims, cfg,
+                     workspace, workspace_bytes, dev_status, stream, 0);
+}
+
+kvarn_status kvarn_decode_attention_append(const void* q, const void* k_new, const void* v_new, void* packed_cache,
+                                           void* scales, void* fp16_tail, const int32_t* block_table,
+                                           const int32_t* seq_lens, void* out, const kvarn_decode_dims* dims,
+                                           const kvarn_config* cfg, void* workspace, size_t workspace_bytes,
+                                           int32_t* dev_status, void* stream) {
+  return decode_impl(q, k_new, v_new, packed_cache, scales, fp16_tail, block_table, seq_lens, out, dims, cfg,
+                     workspace, workspace_bytes, dev_status, stream, 1);
 }
 
 kvarn_status kvarn_decode_attention_noalloc(const void* q, const void* packed_cache, const void* scales,

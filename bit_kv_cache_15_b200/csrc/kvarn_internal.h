@@ -43,6 +43,17 @@ struct DecodeArgs {
   int tiles_per_split, num_splits;
   float sm_scale;
   int32_t* status;
+  // decode step with append (append = 1): seq_lens are the lengths before the
+  // step; each (seq, KV head) first takes k_new / v_new ([B][Hkv][128]) as its
+  // token at position seq_len, written to the fp16 tail; a tail that this
+  // fills (128 tokens) is quantised into block block_table[seq][seq_len / 128]
+  int append;
+  const __half* k_new;
+  const __half* v_new;
+  __half* tail_w;       // the same buffers as tail / packed / scales, written
+  uint8_t* packed_w;
+  uint8_t* scales_w;
+  int iters;
 };
 
 // Split-K geometry: a pure function of the dims (never of seq_lens).

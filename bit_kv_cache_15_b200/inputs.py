@@ -137,6 +137,32 @@ def make_decode_workload(name: str, seq_lens, num_q_heads: int, num_kv_heads: in
                           seq_lens, block_table, slot_mapping, k_full, v_full, tail, q, seed)
 
 
+def append_step(w: DecodeWorkload, seed: int) -> tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """Inputs of one decode step with append on workload w: (k_new, v_new,
+    block_table).  k_new / v_new [B][Hkv][128] fp16 are each sequence's new
+    token (same generators and outlier channels as the workload's K and V).
+    The block table is w's, plus a free pool block (one no full tile uses,
+    in shuffled order) at entry seq_len // 128 of every sequence whose tail
+    the token fills (seq_len % 128 == 127)."""
+    B, hkv = w.num_seqs, w.num_kv_heads
+    outl = pick_outlier_channels(_rng(w.seed, 2), hkv)
+    r = _rng(seed, 7)
+    k_new = gen_k(r, B, hkv, outl)          # one token per sequence: [B][Hkv][128]
+    v_new = gen_v(r, B, hkv)
+    bt = w.block_table.copy()
+    used = set()
+    for b in range(B):
+        used.update(int(x) for x in bt[b, :int(w.seq_lens[b]) // TILE])
+    free = [int(x) for x in r.permutation(w.num_blocks) if int(x) not in used]
+    for b in range(B):
+        L = int(w.seq_lens[b])
+        if L % TILE == TILE - 1:
+            if L // TILE >= bt.shape[1] or not free:
+                raise ValueError("no block-table entry or free block for the filled tile")
+            bt[b, L // TILE] = free.pop()
+    return k_new, v_new, bt
+
+
 # ---------------------------------------------------------------------------
 # The named workloads (sizes as given for the pages' Llama/Qwen shapes)
 # ---------------------------------------------------------------------------

@@ -63,6 +63,8 @@ _SIGS = {
                                      ctypes.POINTER(Config), _vp, _sz, _vp, _vp]),
     "kvarn_decode_attention_noalloc": (_st, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(DecodeDims),
                                              ctypes.POINTER(Config), _vp, _vp]),
+    "kvarn_decode_attention_append": (_st, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(DecodeDims),
+                                            ctypes.POINTER(Config), _vp, _sz, _vp, _vp]),
     "kvarn_baseline_workspace_bytes": (_sz, [ctypes.POINTER(DecodeDims)]),
     "kvarn_decode_attention_fp16": (_st, [_vp, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(DecodeDims),
                                           ctypes.c_float, _vp, _sz, _vp, _vp]),
@@ -197,6 +199,41 @@ def decode_attention(q: torch.Tensor, packed_cache: torch.Tensor, scales: torch.
                                      _ptr(workspace), workspace.numel() * workspace.element_size(),
                                      _ptr(dev_status), _stream(stream))
     _check("kvarn_decode_attention", st)
+    return out
+
+
+def decode_attention_append(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor, packed_cache: torch.Tensor,
+                            scales: torch.Tensor, fp16_tail: torch.Tensor, block_table: torch.Tensor,
+                            seq_lens: torch.Tensor, cfg: Config, out: torch.Tensor | None = None,
+                            workspace: torch.Tensor | None = None, dev_status: torch.Tensor | None = None,
+                            stream=None) -> torch.Tensor:
+    """One decode step with append (kvarn_decode_attention_append in
+    include/kvarn.h): k_new / v_new [B][Hkv][128] fp16 are the step's tokens,
+    seq_lens the lengths before the step (left unchanged: add 1 afterwards).
+    Writes the tail, quantises tails that fill, returns out [B][Hq][128]."""
+    _need(q, "q", torch.float16)
+    _need(k_new, "k_new", torch.float16)
+    _need(v_new, "v_new", torch.float16)
+    _need(packed_cache, "packed_cache", torch.uint8)
+    _need(scales, "scales", torch.uint8)
+    _need(fp16_tail, "fp16_tail", torch.float16)
+    _need(block_table, "block_table", torch.int32)
+    _need(seq_lens, "seq_lens", torch.int32)
+    B, Hq, _ = q.shape
+    Hkv = int(packed_cache.shape[1])
+    if tuple(k_new.shape) != (B, Hkv, 128) or tuple(v_new.shape) != (B, Hkv, 128):
+        raise ValueError("k_new / v_new must be [B][Hkv][128]")
+    d = dims(B, Hq, Hkv, int(block_table.shape[1]), int(packed_cache.shape[0]))
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = torch.zeros(decode_workspace_bytes(cfg, d), dtype=torch.uint8, device=q.device)
+    st = _lib.kvarn_decode_attention_append(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(packed_cache), _ptr(scales),
+                                            _ptr(fp16_tail), _ptr(block_table), _ptr(seq_lens), _ptr(out),
+                                            ctypes.byref(d), ctypes.byref(cfg), _ptr(workspace),
+                                            workspace.numel() * workspace.element_size(), _ptr(dev_status),
+                                            _stream(stream))
+    _check("kvarn_decode_attention_append", st)
     return out
 
 

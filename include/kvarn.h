@@ -165,6 +165,39 @@ KVARN_API kvarn_status kvarn_decode_attention(const void* q, const void* packed_
                                     void* workspace, size_t workspace_bytes,
                                     int32_t* dev_status, void* stream);
 
+/* One decode step that first appends each sequence's new token: the step
+ * before the path in a serving loop (the cache grows by one token per
+ * sequence per step).  The pages keep the newest tokens of a sequence
+ * unquantised until a whole 128-token tile exists and then quantise that tile
+ * ([lehuy] Cơ chế hoạt động: fixed 128-token tiles; [hypho] 需要关注的几个问题
+ * item 3: block size 128); this call does both in the decode kernel.
+ *
+ *  k_new, v_new  fp16 [B][Hkv][128]: the step's token of sequence b.
+ *  seq_lens      int32 [B]: lengths BEFORE the step (L).  The call does not
+ *                change them: the caller adds 1 afterwards.
+ *  fp16_tail, packed_cache, scales   read and written (see below).
+ *  Other arguments as kvarn_decode_attention; workspace size is the same.
+ * For each sequence b and KV head h:
+ *  - the output attends L + 1 tokens: the full tiles i < L/128 from the
+ *    packed cache and rows [0, L % 128] of the fp16 tail, where row L % 128
+ *    is the new token (read from k_new / v_new);
+ *  - the new token is written to row L % 128 of the fp16 tail;
+ *  - if L % 128 == 127 (the tail is now a full tile), the tail tile is
+ *    quantised exactly as kvarn_quantize_tiles would (same config and
+ *    iterations) into block block_table[b][L / 128] (codes and scale records
+ *    of head h).  That block must not be read by any sequence in the same
+ *    call.  After the caller sets seq_len = L + 1, the next call reads that
+ *    tile from the packed cache and the tail is empty.
+ * Requires L + 1 <= 128 * max_blocks_per_seq (else KVARN_DEV_BAD_SEQ_LEN,
+ * output 0, nothing written for b); a block id outside [0, num_blocks) for
+ * the filled tile is reported as KVARN_DEV_BAD_BLOCK and nothing is quantised. */
+KVARN_API kvarn_status kvarn_decode_attention_append(const void* q, const void* k_new, const void* v_new,
+                                                     void* packed_cache, void* scales, void* fp16_tail,
+                                                     const int32_t* block_table, const int32_t* seq_lens, void* out,
+                                                     const kvarn_decode_dims* dims, const kvarn_config* cfg,
+                                                     void* workspace, size_t workspace_bytes,
+                                                     int32_t* dev_status, void* stream);
+
 /* Size of the fixed device scratch used by kvarn_decode_attention_noalloc. */
 #define KVARN_NOALLOC_SCRATCH_BYTES (8u << 20)
 

@@ -294,10 +294,14 @@ def read_tile(packed, scales, blk: int, h: int, side: str, kb: int, vb: int):
 # ---------------------------------------------------------------------------
 
 def gather_kv(packed, scales, tail, block_table, seq_len: int, b: int, h: int, kb: int, vb: int,
-              cache=None):
-    """Explicitly dequantised K, V ([seq_len][128] fp64) of sequence b, head h."""
-    n_full = seq_len // TILE
-    tl = seq_len % TILE
+              cache=None, tail_len=None):
+    """Explicitly dequantised K, V ([seq_len][128] fp64) of sequence b, head h.
+
+    The last `tail_len` tokens (default seq_len % 128) come from the fp16
+    tail, the ones before from the packed cache."""
+    tl = seq_len % TILE if tail_len is None else int(tail_len)
+    assert 0 <= tl <= TILE and (seq_len - tl) % TILE == 0
+    n_full = (seq_len - tl) // TILE
     ks, vs = [], []
     for i in range(n_full):
         blk = int(block_table[b][i])
@@ -348,6 +352,49 @@ def decode(q, packed, scales, tail, block_table, seq_lens, num_kv_heads: int, kb
         K, V = gather_kv(packed, scales, tail, block_table, int(seq_lens[b]), b, h, kb, vb, cache)
         out[b, j] = attention(q[b, j], K, V, sm_scale).astype(np.float16)
     return out
+
+
+def decode_append(q, k_new, v_new, packed, scales, tail, block_table, seq_lens, num_kv_heads: int,
+                  kb: int, vb: int, iters: int = 8, sm_scale: float | None = None, heads=None):
+    """One decode step that first appends each sequence's new token.
+
+    Reading (the pages fix only that whole 128-token tiles are quantised
+    [lehuy, Cơ chế hoạt động; hypho, 需要关注的几个问题 item 3]): the newest
+    seq_len % 128 tokens wait unquantised in the fp16 tail; the step's token
+    (k_new / v_new [B][Hkv][128] fp16) becomes tail row L % 128, where L =
+    seq_lens[b] is the length before the step; the output attends all L + 1
+    tokens, the tail rows [0, L % 128] in fp16; a tail that the token fills
+    is attended in fp16 this step and quantised (quantize_tile, as on write)
+    into block block_table[b][L // 128] for the steps after.
+
+    Returns (out, packed, scales, tail), the last three as new arrays.
+    """
+    B, Hq, _ = q.shape
+    G = Hq // num_kv_heads
+    if sm_scale is None:
+        sm_scale = 1.0 / np.sqrt(HEAD_DIM)
+    tail2, packed2, scales2 = tail.copy(), packed.copy(), scales.copy()
+    for b in range(B):
+        L = int(seq_lens[b])
+        r = L % TILE
+        tail2[b, 0, :, r, :] = k_new[b]
+        tail2[b, 1, :, r, :] = v_new[b]
+        if r == TILE - 1:
+            blk = int(block_table[b][L // TILE])
+            for h in range(num_kv_heads):
+                for sidx, side, bits, off in ((0, "K", kb, 0), (1, "V", vb, side_bytes(kb))):
+                    t = quantize_tile(np.ascontiguousarray(tail2[b, sidx, h]), bits, iters)
+                    packed2[blk, h, off:off + side_bytes(bits)] = pack_codes(t["codes"], side, bits)
+                    scales2[blk, h, sidx] = pack_scales(t["Lt"], t["Lc"], t["zero"], t["step"])
+    out = np.zeros((B, Hq, HEAD_DIM), dtype=np.float16)
+    pairs = heads if heads is not None else [(b, j) for b in range(B) for j in range(Hq)]
+    cache = {}
+    for b, j in pairs:
+        h = j // G
+        L = int(seq_lens[b])
+        K, V = gather_kv(packed, scales, tail2, block_table, L + 1, b, h, kb, vb, cache, tail_len=L % TILE + 1)
+        out[b, j] = attention(q[b, j], K, V, sm_scale).astype(np.float16)
+    return out, packed2, scales2, tail2
 
 
 def decode_folded(q, packed, scales, tail, block_table, seq_lens, num_kv_heads: int, kb: int, vb: int,

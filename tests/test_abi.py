@@ -123,3 +123,18 @@ def test_binding_fails_loudly_without_library(tmp_path):
     r = subprocess.run([sys.executable, "-c", "import bit_kv_cache_15_b200.kvarn"], cwd=tmp_path,
                        capture_output=True, text=True)
     assert r.returncode != 0 and "libkvarn.so is missing" in r.stderr
+
+
+def test_decode_append_argument_checks():
+    cfg = K.config()
+    d = K.dims(2, 8, 2, 4, 16)
+    need = K.decode_workspace_bytes(cfg, d)
+
+    def call(k_new=FAKE, v_new=FAKE, ws_bytes=need, dd=d):
+        return K.lib.kvarn_decode_attention_append(FAKE, k_new, v_new, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                                   ctypes.byref(dd), ctypes.byref(cfg), FAKE, ws_bytes, None, None)
+
+    assert call(k_new=None) == 1
+    assert call(v_new=FAKE + 4) == 1                   # misaligned
+    assert call(ws_bytes=need - 1) == 4
+    assert call(dd=K.dims(0, 8, 2, 4, 16)) == 0         # empty batch: nothing to do

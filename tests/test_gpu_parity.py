@@ -71,65 +71,73 @@ def _fp16_neighbours_ok(gpu16, x64, tol=LOG_TOL):
     return (g >= lo) & (g <= hi)
 
 
+def check_tile(x, bits, codes, Lt, Lc, zero, step, cnt, lt_gpu=None, lc_gpu=None, where=()):
+    """Stages 1-4 for one tile x ([128][128] fp16) against the GPU's stored
+    codes / Lt / Lc / zero / step (stage 1 only with the GPU's fp32
+    log-scales).  Adds counts to cnt."""
+    r = O.quantize_tile(x, bits, 8)
+    if lt_gpu is not None:   # stage 1
+        e1 = np.max(np.abs(lt_gpu - r["lt"]))
+        e2 = np.max(np.abs(lc_gpu - r["lc"]))
+        cnt["worst_scale"] = max(cnt.get("worst_scale", 0.0), e1, e2)
+        assert e1 <= LOG_TOL and e2 <= LOG_TOL, (where, e1, e2)
+    # stage 2
+    assert np.all(_fp16_neighbours_ok(Lt, r["lt"])), where
+    assert np.all(_fp16_neighbours_ok(Lc, r["lc"])), where
+    # stage 3: codes given the GPU's stored scales, zero and step
+    R32 = r["R"].astype(np.float32)
+    c_given, z2, s2, y = O.quantize_given_scales(R32, Lt, Lc, bits)
+    assert abs(float(z2) - float(zero)) <= 1e-6 * max(1.0, abs(float(zero))) + 1e-30, (z2, zero)
+    assert abs(float(s2) - float(step)) <= 1e-6 * float(s2), (s2, step)
+    c_g, _, _, y_g = O.quantize_given_scales(R32, Lt, Lc, bits, zero, step)
+    diff = codes != c_g
+    if diff.any():
+        assert np.all(np.abs(codes[diff] - c_g[diff]) == 1)
+        mt = O.multipliers(Lt).astype(np.float64)[:, None]
+        mc = O.multipliers(Lc).astype(np.float64)[None, :]
+        dR = 2.0 ** -18 * np.abs(x.astype(np.float64)).sum(axis=1)[:, None]
+        dy = dR * mt * mc / float(step) + 2.0 ** -20 * np.abs(y_g)
+        frac = np.abs(y_g - np.floor(y_g) - 0.5)
+        assert np.all(frac[diff] <= dy[diff]), (where, frac[diff].max())
+    # stage 4: end to end.  Where a stored scale (or the tile's grid)
+    # legitimately differs from the oracle's at a rounding boundary, stage 3
+    # has already validated the codes; the unique part is the elements whose
+    # scales and grid agree.
+    e2e = codes != r["codes"]
+    same = (Lt == r["Lt"])[:, None] & (Lc == r["Lc"])[None, :]
+    if not (zero == r["zero"] and step == r["step"]):
+        same[:] = False
+    for k, v in (("mism_given", int(diff.sum())), ("mism_e2e", int(e2e.sum())), ("total", codes.size),
+                 ("mism_same", int((e2e & same).sum())), ("total_same", int(same.sum()))):
+        cnt[k] = cnt.get(k, 0) + v
+
+
+def assert_counts(cnt, kb, vb):
+    assert cnt["mism_same"] <= 1e-4 * cnt["total_same"], cnt
+    if max(kb, vb) <= 4:
+        assert cnt["mism_e2e"] <= 1e-4 * cnt["total"], cnt
+
+
 def check_quantize_parity(K, k, v, slot, num_blocks, kb, vb, groups=None, report=None):
     packed, scales, dbg = gpu_quantize(K, k, v, slot, num_blocks, f"kvarn_k{kb}v{vb}_g128")
     hkv = k.shape[1]
     n_groups = k.shape[0] // 128
     groups = range(n_groups) if groups is None else groups
-    total = mism_e2e = mism_given = total_same = mism_same = 0
-    worst_scale = 0.0
+    cnt = {}
     for g in groups:
         blk = int(slot[g * 128]) // 128
         for h in range(hkv):
             for side, src, bits in (("K", k, kb), ("V", v, vb)):
                 x = np.ascontiguousarray(src[g * 128:(g + 1) * 128, h, :])
-                r = O.quantize_tile(x, bits, 8)
                 codes, Lt, Lc, zero, step = O.read_tile(packed, scales, blk, h, side, kb, vb)
                 sidx = 0 if side == "K" else 1
-                lt_gpu = dbg[g, h, sidx, :128].astype(np.float64)
-                lc_gpu = dbg[g, h, sidx, 128:].astype(np.float64)
-                # stage 1
-                e1 = np.max(np.abs(lt_gpu - r["lt"]))
-                e2 = np.max(np.abs(lc_gpu - r["lc"]))
-                worst_scale = max(worst_scale, e1, e2)
-                assert e1 <= LOG_TOL and e2 <= LOG_TOL, (g, h, side, e1, e2)
-                # stage 2
-                assert np.all(_fp16_neighbours_ok(Lt, r["lt"])), (g, h, side)
-                assert np.all(_fp16_neighbours_ok(Lc, r["lc"])), (g, h, side)
-                # stage 3: codes given the GPU's stored scales, zero and step
-                R32 = r["R"].astype(np.float32)
-                c_given, z2, s2, y = O.quantize_given_scales(R32, Lt, Lc, bits)
-                assert abs(float(z2) - float(zero)) <= 1e-6 * max(1.0, abs(float(zero))) + 1e-30, (z2, zero)
-                assert abs(float(s2) - float(step)) <= 1e-6 * float(s2), (s2, step)
-                c_g, _, _, y_g = O.quantize_given_scales(R32, Lt, Lc, bits, zero, step)
-                diff = codes != c_g
-                if diff.any():
-                    assert np.all(np.abs(codes[diff] - c_g[diff]) == 1)
-                    mt = O.multipliers(Lt).astype(np.float64)[:, None]
-                    mc = O.multipliers(Lc).astype(np.float64)[None, :]
-                    dR = 2.0 ** -18 * np.abs(x.astype(np.float64)).sum(axis=1)[:, None]
-                    dy = dR * mt * mc / float(step) + 2.0 ** -20 * np.abs(y_g)
-                    frac = np.abs(y_g - np.floor(y_g) - 0.5)
-                    assert np.all(frac[diff] <= dy[diff]), (g, h, side, frac[diff].max())
-                mism_given += int(diff.sum())
-                # stage 4: end to end.  Where a stored scale (or the tile's grid)
-                # legitimately differs from the oracle's at a rounding boundary,
-                # stage 3 has already validated the codes; the unique part is
-                # the elements whose scales and grid agree.
-                e2e = codes != r["codes"]
-                same = (Lt == r["Lt"])[:, None] & (Lc == r["Lc"])[None, :]
-                if not (zero == r["zero"] and step == r["step"]):
-                    same[:] = False
-                mism_e2e += int(e2e.sum())
-                mism_same += int((e2e & same).sum())
-                total += codes.size
-                total_same += int(same.sum())
+                check_tile(x, bits, codes, Lt, Lc, zero, step, cnt,
+                           dbg[g, h, sidx, :128].astype(np.float64), dbg[g, h, sidx, 128:].astype(np.float64),
+                           where=(g, h, side))
     if report is not None:
-        report.update(total=total, mism_e2e=mism_e2e, mism_given=mism_given, worst_scale=worst_scale,
-                      total_same=total_same, mism_same=mism_same)
-    assert mism_same <= 1e-4 * total_same, (mism_same, total_same)
-    if max(kb, vb) <= 4:
-        assert mism_e2e <= 1e-4 * total, (mism_e2e, total)
+        report.update(total=cnt["total"], mism_e2e=cnt["mism_e2e"], mism_given=cnt["mism_given"],
+                      worst_scale=cnt["worst_scale"], total_same=cnt["total_same"], mism_same=cnt["mism_same"])
+    assert_counts(cnt, kb, vb)
     return packed, scales
 
 
@@ -271,6 +279,104 @@ def test_decode_quality_vs_fp16_reported(K):
     rel = np.abs(out.astype(np.float64) - ref).mean() / np.abs(ref).mean()
     print(f"k4v2 vs fp16 attention: mean relative error {rel:.3f}")
     assert rel < 1.0
+
+
+# ------------------------------------------------------------------ decode step with append
+
+APPEND_LENS = [0, 127, 128 + 127, 300, 128, 40 * 128 + 127, 5, 2 * 128]
+
+
+def run_append_case(K, lens, hq, hkv, seed, kb=4, vb=2):
+    """One decode step with append on the GPU against the oracle's step over
+    the GPU's own pre-step cache.  Returns the GPU and oracle results."""
+    full = sum(int(L) // 128 for L in lens)
+    w = inputs.make_decode_workload("append", lens, hq, hkv, seed, pool_blocks=full + 8)
+    k_new, v_new, bt = inputs.append_step(w, seed + 1)
+    cfg = K.config(f"kvarn_k{kb}v{vb}_g128")
+    packed, scales = K.alloc_cache(cfg, w.num_blocks, hkv)
+    if w.k_full.shape[0]:
+        K.quantize_tiles(_dev(w.k_full), _dev(w.v_full), _dev(w.slot_mapping), packed, scales, cfg)
+    torch.cuda.synchronize()
+    p0, s0 = packed.cpu().numpy(), scales.cpu().numpy()
+    tail = _dev(w.tail)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = K.decode_attention_append(_dev(w.q), _dev(k_new), _dev(v_new), packed, scales, tail, _dev(bt),
+                                    _dev(w.seq_lens), cfg, dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    ref, p2, s2, t2 = O.decode_append(w.q, k_new, v_new, p0, s0, w.tail, bt, w.seq_lens, hkv, kb, vb)
+    return dict(w=w, bt=bt, k_new=k_new, v_new=v_new, cfg=cfg, out=out.cpu().numpy(), ref=ref,
+                packed=packed, scales=scales, tail=tail, p0=p0, s0=s0, p2=p2, s2=s2, t2=t2)
+
+
+@pytest.mark.parametrize("G", [1, 8])
+def test_decode_append_parity(K, G):
+    """Lengths before the step cover: empty, a tail filled with no full tile,
+    a fill after full tiles, mid-tile, a tail starting, a long fill.  Output
+    within the decode bound; the tail written bit-exactly; blocks other than
+    the filled ones untouched; filled blocks through the quantiser's stages."""
+    r = run_append_case(K, APPEND_LENS, 2 * G, 2, seed=500 + G)
+    w = r["w"]
+    pairs = [(b, j) for b in range(w.num_seqs) for j in range(w.num_q_heads)]
+    err, bnd, _ = decode_errors(r["out"], r["ref"], pairs)
+    print(f"append G={G}: decode max err {err.max():.2e}")
+    assert np.all(err <= bnd)
+    assert np.array_equal(r["tail"].cpu().numpy(), r["t2"])
+    packed, scales = r["packed"].cpu().numpy(), r["scales"].cpu().numpy()
+    filled = {int(r["bt"][b, L // 128]): b for b, L in enumerate(APPEND_LENS) if L % 128 == 127}
+    others = [i for i in range(w.num_blocks) if i not in filled]
+    assert np.array_equal(packed[others], r["p0"][others]) and np.array_equal(scales[others], r["s0"][others])
+    cnt = {}
+    for blk, b in filled.items():
+        for h in range(w.num_kv_heads):
+            for sidx, side, bits in ((0, "K", 4), (1, "V", 2)):
+                x = np.ascontiguousarray(r["t2"][b, sidx, h])
+                codes, Lt, Lc, zero, step = O.read_tile(packed, scales, blk, h, side, 4, 2)
+                check_tile(x, bits, codes, Lt, Lc, zero, step, cnt, where=(b, h, side))
+    assert cnt["total"] == len(filled) * w.num_kv_heads * 2 * 128 * 128
+    assert_counts(cnt, 4, 2)
+
+
+def test_decode_append_then_next_step(K):
+    """The step after an append (seq_len + 1, plain decode) reads the filled
+    tile from the packed cache: parity against the oracle on the GPU's cache."""
+    r = run_append_case(K, APPEND_LENS, 8, 2, seed=520)
+    w = r["w"]
+    lens1 = (w.seq_lens + 1).astype(np.int32)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = K.decode_attention(_dev(w.q), r["packed"], r["scales"], r["tail"], _dev(r["bt"]), _dev(lens1), r["cfg"],
+                             dev_status=status).cpu().numpy()
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    ref = O.decode(w.q, r["packed"].cpu().numpy(), r["scales"].cpu().numpy(), r["tail"].cpu().numpy(), r["bt"],
+                   lens1, 2, 4, 2)
+    err, bnd, _ = decode_errors(out, ref, [(b, j) for b in range(w.num_seqs) for j in range(8)])
+    assert np.all(err <= bnd)
+
+
+def test_decode_append_status(K):
+    """A step whose token would not fit the block table reports a bad length
+    and leaves that sequence's output 0; a bad block id for a filled tile
+    reports a bad block."""
+    w = inputs.make_decode_workload("append", [128, 127], 2, 1, seed=530, pool_blocks=4, max_blocks_per_seq=2)
+    k_new, v_new, bt = inputs.append_step(w, 531)
+    cfg = K.config()
+    packed, scales = K.alloc_cache(cfg, w.num_blocks, 1)
+    K.quantize_tiles(_dev(w.k_full), _dev(w.v_full), _dev(w.slot_mapping), packed, scales, cfg)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    bt1 = np.ascontiguousarray(bt[:, :1])                 # max_blocks 1: L = 128 has no room
+    out = K.decode_attention_append(_dev(w.q), _dev(k_new), _dev(v_new), packed, scales, _dev(w.tail), _dev(bt1),
+                                    _dev(w.seq_lens), cfg, dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 3                       # KVARN_DEV_BAD_SEQ_LEN
+    assert np.all(out.cpu().numpy()[0] == 0)
+    status.zero_()
+    bt2 = bt.copy()
+    bt2[1, 0] = w.num_blocks + 5                          # the filled tile's block is out of range
+    K.decode_attention_append(_dev(w.q), _dev(k_new), _dev(v_new), packed, scales, _dev(w.tail), _dev(bt2),
+                              _dev(w.seq_lens), cfg, dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 2                       # KVARN_DEV_BAD_BLOCK
 
 
 # ------------------------------------------------------------------ full-size, sampled

@@ -357,3 +357,84 @@ def test_e4m3_codec_against_definition():
     # ties go to the even code: 1 + 1/16 lies halfway between 1 (0x38) and 1.125 (0x39)
     assert O.float_to_e4m3(np.array([1.0625]))[0] == 0x38
     assert O.float_to_e4m3(np.array([1e6]))[0] == 0x7E
+
+
+# ---------------------------------------------------------------------------
+# decode step with append
+# ---------------------------------------------------------------------------
+
+def _append_case(lens, hq, hkv, seed, extra_blocks=4, kb=4, vb=2):
+    full = sum(int(L) // 128 for L in lens)
+    w = inputs.make_decode_workload("append", lens, hq, hkv, seed, pool_blocks=full + extra_blocks)
+    k_new, v_new, bt = inputs.append_step(w, seed + 1)
+    packed, scales = O.quantize_tiles(w.k_full, w.v_full, w.slot_mapping, hkv, w.num_blocks, kb, vb)
+    return w, k_new, v_new, bt, packed, scales
+
+
+def _rows_after_append(w, k_new, v_new, b):
+    """All L + 1 fp16 K / V rows of sequence b ([L+1][Hkv][128]) after the append."""
+    s, e = w.token_range(b)
+    tl = int(w.seq_lens[b]) % 128
+    k = np.concatenate([w.k_full[s:e], w.tail[b, 0, :, :tl].transpose(1, 0, 2), k_new[b][None]])
+    v = np.concatenate([w.v_full[s:e], w.tail[b, 1, :, :tl].transpose(1, 0, 2), v_new[b][None]])
+    return k, v
+
+
+def test_append_to_empty_sequence_returns_the_new_value():
+    """One token: its softmax weight is exactly 1, so the output is v_new."""
+    w, k_new, v_new, bt, packed, scales = _append_case([0, 0, 0], 4, 2, seed=41)
+    out, p2, s2, tail2 = O.decode_append(w.q, k_new, v_new, packed, scales, w.tail, bt, w.seq_lens, 2, 4, 2)
+    for b in range(3):
+        for j in range(4):
+            assert np.array_equal(out[b, j], v_new[b, j // 2])
+    assert np.array_equal(tail2[:, 0, :, 0], k_new) and np.array_equal(tail2[:, 1, :, 0], v_new)
+    assert np.array_equal(p2, packed) and np.array_equal(s2, scales)
+
+
+def test_append_before_any_full_tile_is_textbook_attention():
+    """With no full tile, every token (the one that fills the tile included)
+    is attended in fp16: the output is plain softmax attention over the rows."""
+    lens = [5, 64, 127, 126]
+    w, k_new, v_new, bt, packed, scales = _append_case(lens, 8, 2, seed=43)
+    out, *_ = O.decode_append(w.q, k_new, v_new, packed, scales, w.tail, bt, w.seq_lens, 2, 4, 2)
+    rows = [_rows_after_append(w, k_new, v_new, b) for b in range(len(lens))]
+    ref = O.decode_uncompressed(w.q, [r[0] for r in rows], [r[1] for r in rows], w.seq_lens + 1, 2)
+    assert np.array_equal(out, ref)
+
+
+def test_append_mid_tile_equals_decode_of_the_extended_cache():
+    """A token that does not fill its tile is one more tail row: decode of the
+    cache with seq_len + 1 over the written tail gives the same output."""
+    lens = [300, 129, 256 + 5, 128]
+    w, k_new, v_new, bt, packed, scales = _append_case(lens, 8, 2, seed=45)
+    out, p2, s2, tail2 = O.decode_append(w.q, k_new, v_new, packed, scales, w.tail, bt, w.seq_lens, 2, 4, 2)
+    assert np.array_equal(p2, packed) and np.array_equal(s2, scales)
+    ref = O.decode(w.q, packed, scales, tail2, bt, w.seq_lens + 1, 2, 4, 2)
+    assert np.array_equal(out, ref)
+
+
+def test_append_fill_quantises_the_tile_like_the_write_path():
+    """A token that fills the tail: the tile (127 tail rows + the token) lands
+    in the new block exactly as the quantise-on-write path would put it there,
+    only that block changes, and the output still attends the tile in fp16."""
+    lens = [127, 128 + 127, 300]
+    w, k_new, v_new, bt, packed, scales = _append_case(lens, 4, 2, seed=47, kb=4, vb=2)
+    out, p2, s2, tail2 = O.decode_append(w.q, k_new, v_new, packed, scales, w.tail, bt, w.seq_lens, 2, 4, 2)
+    changed = set()
+    for b, L in enumerate(lens):
+        if L % 128 != 127:
+            continue
+        blk = int(bt[b, L // 128])
+        changed.add(blk)
+        k, v = _rows_after_append(w, k_new, v_new, b)
+        tile_k, tile_v = k[L // 128 * 128:], v[L // 128 * 128:]
+        slot = blk * 128 + np.arange(128, dtype=np.int64)
+        pw, sw = O.quantize_tiles(tile_k, tile_v, slot, 2, w.num_blocks, 4, 2)
+        assert np.array_equal(p2[blk], pw[blk]) and np.array_equal(s2[blk], sw[blk])
+    others = [i for i in range(w.num_blocks) if i not in changed]
+    assert np.array_equal(p2[others], packed[others]) and np.array_equal(s2[others], scales[others])
+    # the filled tile is attended in fp16 this step: the same output as a tail of 128 rows
+    b = 0
+    k, v = _rows_after_append(w, k_new, v_new, b)
+    ref = O.decode_uncompressed(w.q[b:b + 1], [k], [v], np.array([128]), 2)
+    assert np.array_equal(out[b], ref[0])
