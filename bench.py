@@ -377,6 +377,8 @@ def precision_sweep(w, dev, iters=30):
         nbytes = HKV * (n_full_tok // 128 * (2048 * (kb + vb) + 1056) + tail_tok * 512) + 2 * BATCH * HQ * 256
         res[f"k{kb}v{vb}"] = {"us": us, "tokens_per_s": BATCH / (us * 1e-6), "hbm_gbs": nbytes / (us * 1e-6) / 1e9,
                               "bytes": nbytes}
+        if (kb, vb) == (4, 2):
+            res.update(append_step(w, dev, cfg, kf, vf, slot, q, tail, sl, out, ws, nbytes, timed))
         del packed, scales
     # uncompressed caches: full tiles from the same K/V, the tail in one extra block per sequence
     nb = w.num_blocks + BATCH
@@ -405,6 +407,50 @@ def precision_sweep(w, dev, iters=30):
     us = timed(lambda: K.decode_attention_fp8(q, k8, v8, bt2d, sl, k_scale, v_scale, out=out, workspace=wsb))
     nbytes = HKV * (n_full_tok + tail_tok) * 256 + 2 * BATCH * HQ * 256
     res["fp8"] = {"us": us, "tokens_per_s": BATCH / (us * 1e-6), "hbm_gbs": nbytes / (us * 1e-6) / 1e9, "bytes": nbytes}
+    return res
+
+
+def append_step(w, dev, cfg, kf, vf, slot, q, tail, sl, out, ws, decode_bytes, timed):
+    """The decode step with append (k4v2) on the same problem: (a) as the
+    workload stands (its tails are U{0..127}; a sequence at 127 fills), and
+    (b) with every sequence's tail at 127 rows, so each (sequence, KV head)
+    quantises a tile inside the step (the worst case, 64 tiles of K and V).
+    Repeated calls rewrite the same tail row and block, so they are identical."""
+    import torch
+    from bit_kv_cache_15_b200 import kvarn as K
+    g = torch.Generator(device=dev).manual_seed(77)
+    k_new = torch.randn((BATCH, HKV, 128), generator=g, device=dev).half()
+    v_new = torch.randn((BATCH, HKV, 128), generator=g, device=dev).half()
+    lens = [int(x) for x in w.seq_lens]
+    nb = w.num_blocks + BATCH
+    packed, scales = K.alloc_cache(cfg, nb, HKV, device=dev)
+    K.quantize_tiles(kf, vf, slot, packed, scales, cfg)
+    bt = w.block_table.copy()
+    fills = 0
+    for b, L in enumerate(lens):
+        if L % 128 == 127:
+            bt[b, L // 128] = w.num_blocks + b
+            fills += 1
+    btd = torch.from_numpy(bt).to(dev)
+    tl = tail.clone()
+    new_bytes = 2 * BATCH * HKV * 256 * 2          # k_new / v_new read, tail rows written
+    tile_bytes = HKV * (2 * 32768 + 2048 * 6 + 1056)  # per filled sequence: both tiles read, codes + scales written
+    us = timed(lambda: K.decode_attention_append(q, k_new, v_new, packed, scales, tl, btd, sl, cfg, out=out,
+                                                 workspace=ws))
+    res = {"append_k4v2": {"us": us, "tokens_per_s": BATCH / (us * 1e-6), "fills": fills,
+                           "bytes": decode_bytes + new_bytes + fills * tile_bytes}}
+    lens_f = [L // 128 * 128 + 127 for L in lens]
+    bt_f = w.block_table.copy()
+    for b, L in enumerate(lens_f):
+        if L // 128 >= bt_f.shape[1]:
+            return res
+        bt_f[b, L // 128] = w.num_blocks + b
+    btf = torch.from_numpy(bt_f).to(dev)
+    slf = torch.tensor(lens_f, dtype=torch.int32, device=dev)
+    us = timed(lambda: K.decode_attention_append(q, k_new, v_new, packed, scales, tl, btf, slf, cfg, out=out,
+                                                 workspace=ws))
+    res["append_fill_all_k4v2"] = {"us": us, "tokens_per_s": BATCH / (us * 1e-6), "fills": BATCH,
+                                   "quantised_tiles": 2 * BATCH * HKV}
     return res
 
 

@@ -112,8 +112,11 @@ __device__ __forceinline__ float hf(const __half* p, int i) { return __half2floa
 // Quantise the full fp16 tail tile of (b, h) -- rows 0..126 from the tail
 // buffer, row 127 = the appended token -- into block block_table[b][L / 128]
 // (K then V), by the whole CTA, with the rotation recomputed (no tensor memory).
+// Kept out of line: it runs once per 128 steps of a sequence, and inlined its
+// code pushed the split loop out of the instruction cache (no_instruction
+// stalls 0.2 -> 1.75 per issue, decode 60 -> 66 us under ncu).
 template <int KB, int VB>
-__device__ void quantize_full_tail(const DecodeArgs& p, uint8_t* smem, int b, int h, int L) {
+__device__ __noinline__ void quantize_full_tail(const DecodeArgs& p, uint8_t* smem, int b, int h, int L) {
   using namespace qt;
   const int tid = threadIdx.x;
   const int32_t blk = p.block_table[(int64_t)b * p.max_blocks + (L >> 7)];
