@@ -46,13 +46,6 @@ __device__ __forceinline__ uint32_t off16(int t, int c16) {
   return (c16 >> 3) * kHalf16 + t * 128 + (((c16 & 7) ^ (t & 7)) << 4);
 }
 
-__device__ __forceinline__ void ldmatrix_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
-                                              uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
-}
-
 __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t x) {
   uint32_t y;
   asm("cvt.rn.f16x2.e4m3x2 %0, %1;\n" : "=r"(y) : "h"(x));

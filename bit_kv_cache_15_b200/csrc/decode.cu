@@ -11,19 +11,22 @@
 //             p'_t = p_t * 2^Lt_v[t]                            (value side)
 // and the output is (acc H / 128 + tail part) / l.
 //
-// Grid: (num_splits + 1, Hkv, B), 4 warps per CTA.  CTA (s, h, b) with
-// s < num_splits owns tiles [s*T, s*T+T) of sequence b; its warps take them
-// round-robin, each warp running its own online softmax.  Each warp streams
+// Work split (stream-K): every (sequence, KV head) pair contributes its full
+// tiles plus one tail unit; the units, in (sequence, head, tile) order, are
+// cut into equal contiguous ranges, one per CTA of a grid of two CTAs per SM.
+// A CTA decodes each run of one pair's tiles in its range with all 4 warps
+// (units round-robin over the warps, each warp running its own online
+// softmax, merged into one partial record per query head), attends a tail
+// unit in its range exactly in the unrotated domain, and the last CTA to
+// finish a pair merges its records and applies H / 128.  Each warp streams
 // its tiles through a private 2-stage shared-memory ring filled by bulk
 // copies (cp.async.bulk on the TMA engine).  Codes are laid out in the mma
-// fragment order, so a lane's 16-byte shared loads are its operands: a LOP3
-// turns each masked word into an f16x2 of exact small integers and one HFMA2
-// removes the magic offset.  Both contractions run on the tensor cores
-// (mma.m16n8k16, fp32 accumulate): K side rows = tokens, N = the 8 query
-// heads; V side rows = channels, N = heads, with the softmax weights moved
-// from accumulator to operand layout by movmatrix.  CTA s = num_splits
-// attends the fp16 tail (seq_len % 128 tokens) exactly, in the unrotated
-// domain.  A second kernel merges the partials and applies H / 128.
+// fragment order, so a lane's 16-byte shared loads are its operands; each
+// masked code pair is already an f16x2 of exact subnormals.  Both
+// contractions run on the tensor cores (mma.m16n8k16, fp32 accumulate): K
+// side rows = tokens, N = the 8 query heads; V side rows = channels, N =
+// heads, with the softmax weights moved from accumulator to operand layout
+// by movmatrix.
 #include <atomic>
 #include <mutex>
 
@@ -71,6 +74,7 @@ struct DecodeTraits {
   static_assert(kDWarps * kDStages * 8 <= 128, "barrier area");
   // the append path stages a 32 KB fp16 tile and the quantiser scratch below the barriers
   static_assert(kBarOff >= 2 * qt::kBox + static_cast<int>(sizeof(qt::QuantScratch)), "append staging");
+  static_assert(kBarOff >= 8 * 8 * 1024, "tail staging: 8 units of 8 KB");
 };
 
 // Where a code of `slot` sits in its fp16 half-word for the mma: bit
@@ -149,92 +153,163 @@ __device__ __noinline__ void quantize_full_tail(const DecodeArgs& p, uint8_t* sm
   }
 }
 
+// Tail attention (a9) on the tensor cores.  The tail rows (fp16, unrotated)
+// are staged in 16-row units: K then V, each two 64-channel halves of
+// 16 rows x 128 bytes, 16-byte chunks XOR-swizzled by row so ldmatrix reads
+// are conflict-free; rows at or past the tail length are zero.
+constexpr int kTU = 16;                  // tail tokens per mma unit
+constexpr int kTHalf = kTU * 128;        // one 64-channel half of a unit side (2 KB)
+constexpr int kTUnitBytes = 4 * kTHalf;  // K halves, then V halves (8 KB)
+
+__device__ __forceinline__ uint32_t toff(int r, int c16) {
+  return (c16 >> 3) * kTHalf + r * 128 + (((c16 & 7) ^ (r & 7)) << 4);
+}
+
+// The tail of (b, h): seq_len % 128 rows, plus the step's own token when
+// appending (taken from k_new / v_new, also written to the tail buffer; a
+// tail it fills is quantised).  Writes one partial record per query head
+// (original domain) to the tail slots.
 template <int KB, int VB>
-__device__ void decode_tail(const DecodeArgs& p, uint8_t* smem, float* qs, int b, int h, int L) {
+__device__ void decode_tail(const DecodeArgs& p, uint8_t* smem, int b, int h, int L) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  // with append, the step's own token (position L) is the tail's last row and
-  // is read from k_new / v_new; it is also written to the tail buffer
+  const int g8 = lane >> 2, c = lane & 3;
   const int tl = (L & 127) + p.append;
   if (tl == 0) return;
   const int G = p.G;
-  float* sc = reinterpret_cast<float*>(smem);  // [kMaxG][128] scores, then weights
-  for (int g = 0; g < kMaxG; ++g)
-    qs[g * 128 + tid] = g < G ? __half2float(p.q[((int64_t)b * p.Hq + h * G + g) * kHeadDim + tid]) : 0.f;
-  __syncthreads();
-  const float sl = p.sm_scale * kLog2e;
+  const int nun = (tl + kTU - 1) / kTU;
   const __half* kt = p.tail + (((int64_t)b * 2 + 0) * p.Hkv + h) * (int64_t)(kTile * kHeadDim);
   const __half* vt = p.tail + (((int64_t)b * 2 + 1) * p.Hkv + h) * (int64_t)(kTile * kHeadDim);
   // row tl - 1: the appended token, or the tail buffer's own row (never a null pointer)
   const __half* klast = p.append ? p.k_new + ((int64_t)b * p.Hkv + h) * kHeadDim : kt + (int64_t)(tl - 1) * kHeadDim;
   const __half* vlast = p.append ? p.v_new + ((int64_t)b * p.Hkv + h) * kHeadDim : vt + (int64_t)(tl - 1) * kHeadDim;
+
+  // ---- stage rows [0, 16 * nun) with asynchronous 16-byte copies, all in
+  // flight at once; rows at or past tl are zero-filled (no bytes read)
+  for (int idx = tid; idx < nun * kTU * 16; idx += kDThreads) {
+    const int t = idx >> 4, c16 = idx & 15;
+    const bool live = t < tl;
+    const __half* kr = !live ? kt : (t == tl - 1 ? klast : kt + (int64_t)t * kHeadDim);
+    const __half* vr = !live ? vt : (t == tl - 1 ? vlast : vt + (int64_t)t * kHeadDim);
+    const uint32_t ub = smem_u32(smem + (t >> 4) * kTUnitBytes) + toff(t & 15, c16);
+    cp_async16(ub, reinterpret_cast<const uint4*>(kr) + c16, live ? 16 : 0);
+    cp_async16(ub + 2 * kTHalf, reinterpret_cast<const uint4*>(vr) + c16, live ? 16 : 0);
+  }
+  cp_async_wait_all();
+  // q fragments (B operand of q.K): q[g8][16kt + 2c .. +1] and +8; heads >= G are 0
+  uint32_t qb0[8], qb1[8];
   {
-    const int t = tid;
-    float dots[kMaxG];
+    const __half* qp = p.q + ((int64_t)b * p.Hq + h * G + (g8 < G ? g8 : 0)) * kHeadDim;
 #pragma unroll
-    for (int g = 0; g < kMaxG; ++g) dots[g] = 0.f;
-    if (t < tl) {
-      const uint4* row = reinterpret_cast<const uint4*>(t == tl - 1 ? klast : kt + (int64_t)t * kHeadDim);
-#pragma unroll 4
-      for (int c8 = 0; c8 < 16; ++c8) {
-        const uint4 raw = __ldg(row + c8);
-        const __half2* hp = reinterpret_cast<const __half2*>(&raw);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float2 kv = __half22float2(hp[i]);
-          const int d = c8 * 8 + 2 * i;
-#pragma unroll
-          for (int g = 0; g < kMaxG; ++g) dots[g] = fmaf(qs[g * 128 + d], kv.x, fmaf(qs[g * 128 + d + 1], kv.y, dots[g]));
-        }
-      }
+    for (int kt8 = 0; kt8 < 8; ++kt8) {
+      qb0[kt8] = g8 < G ? __ldg(reinterpret_cast<const unsigned int*>(qp + 16 * kt8 + 2 * c)) : 0u;
+      qb1[kt8] = g8 < G ? __ldg(reinterpret_cast<const unsigned int*>(qp + 16 * kt8 + 2 * c + 8)) : 0u;
     }
-#pragma unroll
-    for (int g = 0; g < kMaxG; ++g) sc[g * 128 + t] = t < tl ? dots[g] * sl : -INFINITY;
   }
   __syncthreads();
-  __shared__ float mrow[kMaxG], lrow[kMaxG];
-  for (int g = warp; g < kMaxG; g += kDWarps) {
-    float v[4];
-    float m = -INFINITY;
+
+  // ---- per warp: units warp, warp + 4 with an online softmax (log2 units)
+  const float sl = p.sm_scale * kLog2e;
+  float acc[8][4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      v[i] = sc[g * 128 + lane + 32 * i];
-      m = fmaxf(m, v[i]);
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int r = 0; r < 4; ++r) acc[i][r] = 0.f;
+  float mrun[2] = {-INFINITY, -INFINITY}, lsum[2] = {0.f, 0.f};
+  const int mi = lane >> 3;
+  for (int un = warp; un < nun; un += kDWarps) {
+    const int valid_rows = min(kTU, tl - un * kTU);
+    const uint32_t kb = smem_u32(smem + un * kTUnitBytes), vb = kb + 2 * kTHalf;
+    float S[4] = {0.f, 0.f, 0.f, 0.f};
+    const int arow = (lane & 7) + 8 * (mi & 1);
+#pragma unroll
+    for (int kt8 = 0; kt8 < 8; ++kt8) {
+      uint32_t a0, a1, a2, a3;
+      ldmatrix_x4(kb + toff(arow, 2 * kt8 + (mi >> 1)), a0, a1, a2, a3);
+      mma_f16(S, a0, a1, a2, a3, qb0[kt8], qb1[kt8]);
     }
-    m = warp_max(m);
-    float l = 0.f;
+    // rows g8 and g8 + 8 (tokens), heads 2c and 2c + 1; tokens past the tail masked
+    const bool v0 = g8 < valid_rows, v1 = g8 + 8 < valid_rows;
+    S[0] = v0 ? S[0] * sl : -INFINITY;
+    S[1] = v0 ? S[1] * sl : -INFINITY;
+    S[2] = v1 ? S[2] * sl : -INFINITY;
+    S[3] = v1 ? S[3] * sl : -INFINITY;
+    float mx0 = fmaxf(S[0], S[2]), mx1 = fmaxf(S[1], S[3]);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float e = ex2_fast(v[i] - m);
-      sc[g * 128 + lane + 32 * i] = e;
-      l += e;
+    for (int o = 4; o < 32; o <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
     }
+    const float mn0 = fmaxf(mrun[0], mx0), mn1 = fmaxf(mrun[1], mx1);
+    const float al0 = ex2_fast(mrun[0] - mn0), al1 = ex2_fast(mrun[1] - mn1);
+    mrun[0] = mn0;
+    mrun[1] = mn1;
+    const float p0 = ex2_fast(S[0] - mn0), p1 = ex2_fast(S[1] - mn1);
+    const float p2 = ex2_fast(S[2] - mn0), p3 = ex2_fast(S[3] - mn1);
+    lsum[0] = lsum[0] * al0 + (p0 + p2);
+    lsum[1] = lsum[1] * al1 + (p1 + p3);
+    const uint32_t bv0 = movmatrix_t(pack_f2h2(p0, p1));
+    const uint32_t bv1 = movmatrix_t(pack_f2h2(p2, p3));
+    // P.V: A = V^T (rows channels, k = the unit's 16 tokens) via ldmatrix.trans
+    const int vrow = (lane & 7) + 8 * (mi >> 1);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-    if (lane == 0) {
-      mrow[g] = m;
-      lrow[g] = l;
+    for (int mt = 0; mt < 8; ++mt) {
+      uint32_t a0, a1, a2, a3;
+      ldmatrix_x4_t(vb + toff(vrow, 2 * mt + (mi & 1)), a0, a1, a2, a3);
+      float o[4] = {0.f, 0.f, 0.f, 0.f};
+      mma_f16(o, a0, a1, a2, a3, bv0, bv1);
+      acc[mt][0] = fmaf(acc[mt][0], al0, o[0]);
+      acc[mt][1] = fmaf(acc[mt][1], al1, o[1]);
+      acc[mt][2] = fmaf(acc[mt][2], al0, o[2]);
+      acc[mt][3] = fmaf(acc[mt][3], al1, o[3]);
     }
   }
+#pragma unroll
+  for (int o = 4; o < 32; o <<= 1) {
+    lsum[0] += __shfl_xor_sync(0xffffffffu, lsum[0], o);
+    lsum[1] += __shfl_xor_sync(0xffffffffu, lsum[1], o);
+  }
+  __syncthreads();   // the staged units are dead; the merge area reuses them
+
+  // ---- merge the four warps, write the tail record per head
+  float* mS = reinterpret_cast<float*>(smem);            // [4][8]
+  float* lS = mS + kDWarps * kMaxG;                      // [4][8]
+  float* aS = lS + kDWarps * kMaxG;                      // [4][8][128]
+  if (g8 == 0) {
+    mS[warp * kMaxG + 2 * c] = mrun[0];
+    mS[warp * kMaxG + 2 * c + 1] = mrun[1];
+    lS[warp * kMaxG + 2 * c] = lsum[0];
+    lS[warp * kMaxG + 2 * c + 1] = lsum[1];
+  }
+#pragma unroll
+  for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+    for (int ri = 0; ri < 2; ++ri) {
+      const int d = 16 * mt + g8 + 8 * ri;
+      aS[(warp * kMaxG + 2 * c) * kHeadDim + d] = acc[mt][2 * ri];
+      aS[(warp * kMaxG + 2 * c + 1) * kHeadDim + d] = acc[mt][2 * ri + 1];
+    }
   __syncthreads();
   const int d = tid;
-  float acc[kMaxG];
-#pragma unroll
-  for (int g = 0; g < kMaxG; ++g) acc[g] = 0.f;
-  for (int t = 0; t < tl; ++t) {
-    const __half* vrow = t == tl - 1 ? vlast : vt + (int64_t)t * kHeadDim;
-    const float vv = __half2float(vrow[d]);
-#pragma unroll
-    for (int g = 0; g < kMaxG; ++g) acc[g] = fmaf(sc[g * 128 + t], vv, acc[g]);
-  }
   for (int g = 0; g < G; ++g) {
-    float* rec = p.ws + (((int64_t)b * p.Hq + h * G + g) * (p.num_splits + 1) + p.num_splits) * kPartialFloats;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kDWarps; ++w) M = fmaxf(M, mS[w * kMaxG + g]);
+    float l = 0.f, a = 0.f;
+#pragma unroll
+    for (int w = 0; w < kDWarps; ++w) {
+      const float mw = mS[w * kMaxG + g];
+      const float f = mw == -INFINITY ? 0.f : ex2_fast(mw - M);
+      l = fmaf(f, lS[w * kMaxG + g], l);
+      a = fmaf(f, aS[(w * kMaxG + g) * kHeadDim + d], a);
+    }
+    float* rec = p.ws_tail + (((int64_t)b * p.Hkv + h) * G + g) * kPartialFloats;
     if (d == 0) {
-      rec[0] = mrow[g];
-      rec[1] = lrow[g];
+      rec[0] = M;
+      rec[1] = l;
       rec[2] = 0.f;
       rec[3] = 0.f;
     }
-    rec[4 + d] = acc[g];
+    rec[4 + d] = a;
   }
   if (p.append) {
     const int r = L & 127;
@@ -243,7 +318,7 @@ __device__ void decode_tail(const DecodeArgs& p, uint8_t* smem, float* qs, int b
     kw[d] = klast[d];
     vw[d] = vlast[d];
     if (tl == kTile) {
-      __syncthreads();   // the scores area is reused for the staged tile
+      __syncthreads();   // the merge area is reused for the staged tile
       quantize_full_tail<KB, VB>(p, smem, b, h, L);
     }
   }
@@ -277,10 +352,15 @@ __device__ __forceinline__ bool issue_unit(const DecodeArgs& p, uint8_t* stage_b
   return ok;
 }
 
-// One split: tiles [s*T, s*T + T) of sequence b, KV head h; writes one
-// partial record per query head (or nothing if the split is empty).
+// One segment: full tiles [t_begin, t_end) of sequence b, KV head h, by the
+// whole CTA; writes one partial record per query head at recs + g * 132.
+// Work units (tile, part) go round-robin over the warps starting at warp
+// `woff`, so a CTA that runs several segments keeps its warps level.  `rearm`:
+// the barriers were used by an earlier segment and are invalidated first.
+// Returns false if a copy timed out (the status is set).
 template <int KB, int VB>
-__device__ __forceinline__ void decode_split(const DecodeArgs& p, uint8_t* smem, int b, int h, int s, int L) {
+__device__ __forceinline__ bool decode_segment(const DecodeArgs& p, uint8_t* smem, int b, int h, int t_begin,
+                                               int t_end, int woff, bool rearm, float* recs) {
   using T = DecodeTraits<KB, VB>;
   constexpr int U = T::U, MT = T::MT;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + T::kBarOff);
@@ -289,13 +369,13 @@ __device__ __forceinline__ void decode_split(const DecodeArgs& p, uint8_t* smem,
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = p.G;
-  const int n_full = L >> 7;
-  const int t_begin = s * p.tiles_per_split;
-  const int t_end = min(t_begin + p.tiles_per_split, n_full);
-  if (t_begin >= t_end) return;
+  if (t_begin >= t_end) return true;
 
   if (tid == 0) {
-    for (int i = 0; i < kDWarps * kDStages; ++i) mbar_init(&bars[i], 1);
+    for (int i = 0; i < kDWarps * kDStages; ++i) {
+      if (rearm) mbar_inval(&bars[i]);
+      mbar_init(&bars[i], 1);
+    }
     fence_barrier_init();
   }
 
@@ -373,31 +453,32 @@ __device__ __forceinline__ void decode_split(const DecodeArgs& p, uint8_t* smem,
     for (int r = 0; r < 4; ++r) acc[i][r] = 0.f;
   float mrun[2] = {-INFINITY, -INFINITY}, lsum[2] = {0.f, 0.f};
 
-  // work units of this split: (tile, part), part in [0, U); warp takes every 4th
+  // work units of this segment: (tile, part), part in [0, U); warp takes every 4th from u0
   const int n_units = (t_end - t_begin) * U;
-  const int n_mine = warp < n_units ? (n_units - warp + kDWarps - 1) / kDWarps : 0;
+  const int u0 = (warp - woff + kDWarps) % kDWarps;
+  const int n_mine = u0 < n_units ? (n_units - u0 + kDWarps - 1) / kDWarps : 0;
   uint8_t* stage_base = smem + warp * kDStages * T::kStage;
   uint64_t* my_bars = bars + warp * kDStages;
   const int32_t* btab = p.block_table + (int64_t)b * p.max_blocks;
 
-  bool ok0 = n_mine > 0 ? issue_unit<KB, VB>(p, stage_base, my_bars, 0, warp, btab[t_begin + warp / U], h, lane)
+  bool ok0 = n_mine > 0 ? issue_unit<KB, VB>(p, stage_base, my_bars, 0, u0, btab[t_begin + u0 / U], h, lane)
                         : false;
-  bool ok1 = n_mine > 1 ? issue_unit<KB, VB>(p, stage_base, my_bars, 1, warp + kDWarps,
-                                             btab[t_begin + (warp + kDWarps) / U], h, lane)
+  bool ok1 = n_mine > 1 ? issue_unit<KB, VB>(p, stage_base, my_bars, 1, u0 + kDWarps,
+                                             btab[t_begin + (u0 + kDWarps) / U], h, lane)
                         : false;
   int k_fail = -1;
 
   for (int k = 0; k < n_mine; ++k) {
     const int stg = k & 1;
     // block id of unit k + 2, loaded now so it is in hand when that copy is issued
-    const int32_t blk_next = k + 2 < n_mine ? btab[t_begin + (warp + (k + 2) * kDWarps) / U] : 0;
+    const int32_t blk_next = k + 2 < n_mine ? btab[t_begin + (u0 + (k + 2) * kDWarps) / U] : 0;
     if (!__all_sync(0xffffffffu, mbar_wait_bounded(&my_bars[stg], (k >> 1) & 1))) {
       if (lane == 0) report_status(p.status, KVARN_DEV_TIMEOUT);
       k_fail = k;
       break;
     }
     const bool tile_ok = stg == 0 ? ok0 : ok1;
-    const int part = (warp + k * kDWarps) % U;
+    const int part = (u0 + k * kDWarps) % U;
     const uint8_t* st = stage_base + stg * T::kStage;
     if (tile_ok) {
       const uint8_t* rk = st + T::kUnitK + T::kUnitV;   // K scale record, V record follows
@@ -611,7 +692,7 @@ __device__ __forceinline__ void decode_split(const DecodeArgs& p, uint8_t* smem,
     }
     __syncwarp();
     if (k + 2 < n_mine) {
-      const bool okn = issue_unit<KB, VB>(p, stage_base, my_bars, k + 2, warp + (k + 2) * kDWarps, blk_next, h, lane);
+      const bool okn = issue_unit<KB, VB>(p, stage_base, my_bars, k + 2, u0 + (k + 2) * kDWarps, blk_next, h, lane);
       if (stg == 0) ok0 = okn; else ok1 = okn;
     }
   }
@@ -628,7 +709,7 @@ __device__ __forceinline__ void decode_split(const DecodeArgs& p, uint8_t* smem,
     lsum[0] += __shfl_xor_sync(0xffffffffu, lsum[0], o);
     lsum[1] += __shfl_xor_sync(0xffffffffu, lsum[1], o);
   }
-  __syncthreads();   // all warps are done with their stages
+  const bool failed = __syncthreads_or(k_fail >= 0) != 0;   // all warps are done with their stages
   float* mS = reinterpret_cast<float*>(smem);            // [4][8]
   float* lS = mS + kDWarps * kMaxG;                      // [4][8]
   float* aS = lS + kDWarps * kMaxG;                      // [4][8][128]
@@ -660,7 +741,7 @@ __device__ __forceinline__ void decode_split(const DecodeArgs& p, uint8_t* smem,
       l = fmaf(f, lS[w * kMaxG + g], l);
       a = fmaf(f, aS[(w * kMaxG + g) * kHeadDim + d], a);
     }
-    float* rec = p.ws + (((int64_t)b * p.Hq + h * G + g) * (p.num_splits + 1) + s) * kPartialFloats;
+    float* rec = recs + (int64_t)g * kPartialFloats;
     if (d == 0) {
       rec[0] = M;
       rec[1] = l;
@@ -669,105 +750,291 @@ __device__ __forceinline__ void decode_split(const DecodeArgs& p, uint8_t* smem,
     }
     rec[4 + d] = a;
   }
+  __syncthreads();   // the merge area and the q buffers are free for the next segment
+  return !failed;
+}
+
+// ------------------------------------------------------------------ stream-K geometry
+
+// Work units of each KV head of sequence b: one per full tile, plus
+// kTailUnits for the fp16 tail (which also carries an empty or invalid
+// sequence, so every pair is owned).  The tail, and usually the merge of the
+// pair, fall to the CTA owning the pair's last unit; weighting them as
+// several tiles keeps that CTA's range shorter.
+constexpr int kTailUnits = 9;
+__device__ __forceinline__ int pair_units(int L, bool valid) { return (valid ? (L >> 7) : 0) + kTailUnits; }
+
+__device__ __forceinline__ bool seq_valid(const DecodeArgs& p, int L) {
+  return L >= 0 && L + p.append <= kTile * p.max_blocks;
+}
+
+// CTA i of P owns units [W*i/P, W*(i+1)/P); owner(u) inverts that.
+__device__ __forceinline__ long long sk_begin(long long W, int P, int i) { return W * i / P; }
+__device__ __forceinline__ int sk_owner(long long W, int P, long long u) {
+  return static_cast<int>(((u + 1) * P - 1) / W);
+}
+
+// Warp 0: total units W, and the sequence whose units hold this CTA's first
+// unit with that sequence's first unit.
+__device__ void sk_locate(const DecodeArgs& p, int cta, int P, long long* W_out, int* b_out, long long* ps_out) {
+  const int lane = threadIdx.x & 31;
+  long long mine = 0;
+  for (int b = lane; b < p.B; b += 32) {
+    const int L = p.seq_lens[b];
+    mine += static_cast<long long>(pair_units(L, seq_valid(p, L))) * p.Hkv;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mine += __shfl_xor_sync(0xffffffffu, mine, o);
+  const long long W = mine;
+  const long long u0 = sk_begin(W, P, cta);
+  long long base = 0;
+  int fb = 0;
+  long long fps = 0;
+  for (int b0 = 0; b0 < p.B; b0 += 32) {
+    const int b = b0 + lane;
+    long long v = 0;
+    if (b < p.B) {
+      const int L = p.seq_lens[b];
+      v = static_cast<long long>(pair_units(L, seq_valid(p, L))) * p.Hkv;
+    }
+    long long incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const long long y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const long long first = base + incl - v;
+    const unsigned hit = __ballot_sync(0xffffffffu, b < p.B && u0 >= first && u0 < first + v);
+    if (hit != 0u) {
+      const int l = __ffs(hit) - 1;
+      fb = b0 + l;
+      fps = __shfl_sync(0xffffffffu, first, l);
+      break;
+    }
+    base += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  *W_out = W;
+  *b_out = fb;
+  *ps_out = fps;
 }
 
 // ------------------------------------------------------------------ combine (a10)
 
-// Merge the partials of (b, h) for its G query heads: o = (acc H / 128 + tail) / l.
-// One warp per head; lane owns channels 4*lane .. 4*lane + 3.  Records written
-// by other CTAs are read with ld.global.cg (L2), never through L1.
-__device__ void combine_pair(const DecodeArgs& p, int b, int h, int L, bool valid) {
+// Merge the partials of pair (b, h) for its G query heads:
+// o = (acc H / 128 + tail) / l.  Tile records come from every CTA whose range
+// meets the pair's full tiles [pst, pst + nt) (record slot pair + CTA), the
+// tail record from its own slot.  One warp per head; lane owns channels
+// 4*lane .. 4*lane + 3.  Records written by other CTAs are read with
+// ld.global.cg (L2), never through L1.
+__device__ void combine_pair(const DecodeArgs& p, int b, int h, int L, bool valid, long long pst, int nt,
+                             long long W, int P) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int g = warp; g < p.G; g += kDWarps) {
-    const int j = h * p.G + g;
-    __half* o = p.out + ((int64_t)b * p.Hq + j) * kHeadDim + 4 * lane;
-    if (!valid || L + p.append == 0) {
-      *reinterpret_cast<uint2*>(o) = make_uint2(0u, 0u);
-      continue;
+  const int pair = b * p.Hkv + h;
+  // CTAs whose ranges meet the tiles: owner(pst) .. owner(pst + nt - 1).  With
+  // W >= P every CTA range is non-empty, so each of them wrote a record.
+  const int i_lo = nt > 0 ? sk_owner(W, P, pst) : 0;
+  const int n_rec = nt > 0 ? sk_owner(W, P, pst + nt - 1) - i_lo + 1 : 0;
+  const bool dense = W >= P;
+  const bool has_tail = (L & 127) + p.append != 0;
+  // a warp merges heads warp and warp + 4 together, so one round of L2 loads
+  // serves both (G <= 8)
+  int gh[2];
+  bool hl[2];
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    gh[k] = warp + kDWarps * k;
+    hl[k] = gh[k] < p.G;
+  }
+  if (!hl[0]) return;
+  if (!valid || L + p.append == 0) {
+#pragma unroll
+    for (int k = 0; k < 2; ++k)
+      if (hl[k]) {
+        __half* o = p.out + ((int64_t)b * p.Hq + h * p.G + gh[k]) * kHeadDim + 4 * lane;
+        *reinterpret_cast<uint2*>(o) = make_uint2(0u, 0u);
+      }
+    return;
+  }
+  float M[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f}, a[2][4];
+  float mt[2], lt[2];
+  float4 vt[2];
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) a[k][i] = 0.f;
+    const float* trec = p.ws_tail + ((int64_t)pair * p.G + (hl[k] ? gh[k] : 0)) * kPartialFloats;
+    const bool t = has_tail && hl[k];
+    mt[k] = t ? __ldcg(trec) : -INFINITY;
+    lt[k] = t ? __ldcg(trec + 1) : 0.f;
+    vt[k] = t ? __ldcg(reinterpret_cast<const float4*>(trec + 4 + 4 * lane)) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  constexpr int kChunk = 8;
+  for (int k0 = 0; k0 < n_rec; k0 += kChunk) {
+    float mr[2][kChunk], lr[2][kChunk];
+    float4 vr[2][kChunk];
+#pragma unroll
+    for (int q = 0; q < kChunk; ++q) {
+      const int i = i_lo + k0 + q;
+      bool live = k0 + q < n_rec;
+      if (live && !dense) live = max(sk_begin(W, P, i), pst) < min(sk_begin(W, P, i + 1), pst + nt);
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const bool lk = live && hl[k];
+        const float* r = p.ws + ((int64_t)(pair + (lk ? i : i_lo)) * p.G + (hl[k] ? gh[k] : 0)) * kPartialFloats;
+        mr[k][q] = lk ? __ldcg(r) : -INFINITY;
+        lr[k][q] = lk ? __ldcg(r + 1) : 0.f;
+        vr[k][q] = lk ? __ldcg(reinterpret_cast<const float4*>(r + 4 + 4 * lane)) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
     }
-    const int n_full = L >> 7;
-    const int nsv = (n_full + p.tiles_per_split - 1) / p.tiles_per_split;
-    const bool has_tail = (L & 127) + p.append != 0;
-    const float* rec = p.ws + ((int64_t)b * p.Hq + j) * (p.num_splits + 1) * kPartialFloats;
-    const float* trec = rec + (int64_t)p.num_splits * kPartialFloats;
-    float M = has_tail ? __ldcg(trec) : -INFINITY;
-    for (int s = 0; s < nsv; ++s) M = fmaxf(M, __ldcg(rec + (int64_t)s * kPartialFloats));
-    float l = 0.f, a[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int s = 0; s < nsv; ++s) {
-      const float* r = rec + (int64_t)s * kPartialFloats;
-      const float w = ex2_fast(__ldcg(r) - M);
-      l = fmaf(w, __ldcg(r + 1), l);
-      const float4 v = __ldcg(reinterpret_cast<const float4*>(r + 4 + 4 * lane));
-      a[0] = fmaf(w, v.x, a[0]);
-      a[1] = fmaf(w, v.y, a[1]);
-      a[2] = fmaf(w, v.z, a[2]);
-      a[3] = fmaf(w, v.w, a[3]);
-    }
+#pragma unroll
+    for (int q = 0; q < kChunk; ++q)
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        if (mr[k][q] == -INFINITY) continue;
+        const float Mn = fmaxf(M[k], mr[k][q]);
+        const float fo = ex2_fast(M[k] - Mn), fr = ex2_fast(mr[k][q] - Mn);
+        l[k] = fmaf(l[k], fo, lr[k][q] * fr);
+        a[k][0] = fmaf(a[k][0], fo, vr[k][q].x * fr);
+        a[k][1] = fmaf(a[k][1], fo, vr[k][q].y * fr);
+        a[k][2] = fmaf(a[k][2], fo, vr[k][q].z * fr);
+        a[k][3] = fmaf(a[k][3], fo, vr[k][q].w * fr);
+        M[k] = Mn;
+      }
+  }
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    if (!hl[k]) continue;
+    float* ak = a[k];
     {   // acc H / 128
-      const float b0 = a[0] + a[1], b1 = a[0] - a[1], b2 = a[2] + a[3], b3 = a[2] - a[3];
-      a[0] = b0 + b2; a[1] = b1 + b3; a[2] = b0 - b2; a[3] = b1 - b3;
+      const float b0 = ak[0] + ak[1], b1 = ak[0] - ak[1], b2 = ak[2] + ak[3], b3 = ak[2] - ak[3];
+      ak[0] = b0 + b2; ak[1] = b1 + b3; ak[2] = b0 - b2; ak[3] = b1 - b3;
 #pragma unroll
       for (int m = 1; m < 32; m <<= 1) {
         const bool up = (lane & m) != 0;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const float y = __shfl_xor_sync(0xffffffffu, a[i], m);
-          a[i] = up ? (y - a[i]) : (a[i] + y);
+          const float y = __shfl_xor_sync(0xffffffffu, ak[i], m);
+          ak[i] = up ? (y - ak[i]) : (ak[i] + y);
         }
       }
 #pragma unroll
-      for (int i = 0; i < 4; ++i) a[i] *= (1.f / 128.f);
+      for (int i = 0; i < 4; ++i) ak[i] *= (1.f / 128.f);
     }
-    if (has_tail) {
-      const float w = ex2_fast(__ldcg(trec) - M);
-      l = fmaf(w, __ldcg(trec + 1), l);
-      const float4 v = __ldcg(reinterpret_cast<const float4*>(trec + 4 + 4 * lane));
-      a[0] = fmaf(w, v.x, a[0]);
-      a[1] = fmaf(w, v.y, a[1]);
-      a[2] = fmaf(w, v.z, a[2]);
-      a[3] = fmaf(w, v.w, a[3]);
+    if (has_tail) {   // the tail, in the original domain
+      const float Mn = fmaxf(M[k], mt[k]);
+      const float fo = ex2_fast(M[k] - Mn), fr = ex2_fast(mt[k] - Mn);
+      l[k] = fmaf(l[k], fo, lt[k] * fr);
+      ak[0] = fmaf(ak[0], fo, vt[k].x * fr);
+      ak[1] = fmaf(ak[1], fo, vt[k].y * fr);
+      ak[2] = fmaf(ak[2], fo, vt[k].z * fr);
+      ak[3] = fmaf(ak[3], fo, vt[k].w * fr);
     }
-    const float il = 1.f / l;
-    const __half2 o01 = __floats2half2_rn(a[0] * il, a[1] * il);
-    const __half2 o23 = __floats2half2_rn(a[2] * il, a[3] * il);
+    const float il = 1.f / l[k];
+    const __half2 o01 = __floats2half2_rn(ak[0] * il, ak[1] * il);
+    const __half2 o23 = __floats2half2_rn(ak[2] * il, ak[3] * il);
+    __half* o = p.out + ((int64_t)b * p.Hq + h * p.G + gh[k]) * kHeadDim + 4 * lane;
     *reinterpret_cast<uint2*>(o) = make_uint2(h2_as_u32(o01), h2_as_u32(o23));
   }
 }
 
-// Grid (num_splits + 1, Hkv, B).  Every CTA of (b, h) -- empty splits and the
-// tail CTA included -- bumps the pair's counter (cleared before the launch)
-// once after its records are visible; the last of the num_splits + 1 arrivals
-// merges them.  Nothing waits on anything.
+// ------------------------------------------------------------------ main kernel
+
+// Stream-K: CTA `cta` of P walks its unit range [W*cta/P, W*(cta+1)/P) pair by
+// pair.  For each pair it meets it decodes the run of full tiles in its range
+// (one partial record per query head, slot pair + cta), attends the tail if
+// the pair's tail unit is in its range, then adds the number of units it did
+// to the pair's counter (cleared before the launch).  The CTA that brings the
+// counter to the pair's unit count merges the pair.  Nothing waits on anything.
 template <int KB, int VB>
 __global__ void __launch_bounds__(kDThreads, KVARN_D_MIN_CTAS) decode_kernel(const __grid_constant__ DecodeArgs p) {
   extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ int last_arrival;
-  const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int L = p.seq_lens[b];   // before the step's own token when appending
-  const bool valid = L >= 0 && L + p.append <= kTile * p.max_blocks;
-  if (!valid) {
-    if (threadIdx.x == 0 && s == 0) report_status(p.status, KVARN_DEV_BAD_SEQ_LEN);
-  } else if (s == p.num_splits) {
-    decode_tail<KB, VB>(p, smem, reinterpret_cast<float*>(smem + DecodeTraits<KB, VB>::kQrotOff), b, h, L);
-  } else {
-    decode_split<KB, VB>(p, smem, b, h, s, L);
+  // walker state (thread 0) and the current segment, in shared memory so that
+  // almost nothing of the walk is live in registers across a segment
+  __shared__ long long sh_W, sh_u, sh_ps, sg_pst;
+  __shared__ int sh_b, sg_b, sg_h, sg_L, sg_nu, sg_ta, sg_te, sg_done, sg_tail, sh_last;
+  const int tid = threadIdx.x, cta = blockIdx.x, P = gridDim.x;
+  if (tid < 32) {
+    long long W, ps;
+    int b0;
+    sk_locate(p, cta, P, &W, &b0, &ps);
+    if (tid == 0) {
+      sh_W = W;
+      sh_u = sk_begin(W, P, cta);
+      sh_b = b0;
+      sh_ps = ps;
+    }
   }
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    int* cnt = p.counters + (int64_t)b * p.Hkv + h;
-    last_arrival = atomicAdd(cnt, 1) == p.num_splits;
+  int woff = 0;
+  bool rearm = false, ok = true;
+  for (;;) {
+    __syncthreads();
+    if (tid == 0) {   // the next segment: one pair's part of this CTA's range
+      const long long W = sh_W, u = sh_u, u_end = sk_begin(W, P, cta + 1);
+      if (u >= u_end) {
+        sg_b = -1;
+      } else {
+        int b = sh_b;
+        long long ps = sh_ps;
+        int L = p.seq_lens[b];
+        int nu = pair_units(L, seq_valid(p, L));
+        if (u >= ps + static_cast<long long>(nu) * p.Hkv) {   // next sequence (each has >= Hkv units)
+          ps += static_cast<long long>(nu) * p.Hkv;
+          ++b;
+          L = p.seq_lens[b];
+          nu = pair_units(L, seq_valid(p, L));
+          sh_b = b;
+          sh_ps = ps;
+        }
+        const int h = static_cast<int>((u - ps) / nu);
+        const long long pst = ps + static_cast<long long>(h) * nu;
+        const long long e = min(u_end, pst + nu);
+        sg_b = b;
+        sg_h = h;
+        sg_L = L;
+        sg_nu = nu;
+        sg_pst = pst;
+        sg_ta = static_cast<int>(u - pst);
+        sg_te = static_cast<int>(min(e - pst, static_cast<long long>(nu - kTailUnits)));
+        sg_tail = e == pst + nu;
+        sg_done = static_cast<int>(e - u);
+        sh_u = e;
+      }
+    }
+    __syncthreads();
+    const int b = sg_b;
+    if (b < 0) break;
+    const int h = sg_h, L = sg_L, t_a = sg_ta, t_e = sg_te;
+    const int pair = b * p.Hkv + h;
+    if (ok && t_a < t_e) {
+      ok = decode_segment<KB, VB>(p, smem, b, h, t_a, t_e, woff, rearm,
+                                  p.ws + static_cast<int64_t>(pair + cta) * p.G * kPartialFloats);
+      rearm = true;
+      woff = (woff + (t_e - t_a) * DecodeTraits<KB, VB>::U) % kDWarps;
+    }
+    if (sg_tail) {   // the pair's tail unit
+      if (!seq_valid(p, L)) {
+        if (tid == 0 && h == 0) report_status(p.status, KVARN_DEV_BAD_SEQ_LEN);
+      } else {
+        decode_tail<KB, VB>(p, smem, b, h, L);
+      }
+      __syncthreads();   // shared memory is free again
+    }
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) sh_last = atomicAdd(p.counters + pair, sg_done) + sg_done == sg_nu;
+    __syncthreads();
+    if (sh_last) {
+      __threadfence();
+      combine_pair(p, b, h, L, seq_valid(p, L), sg_pst, sg_nu - kTailUnits, sh_W, P);
+    }
   }
-  __syncthreads();
-  if (!last_arrival) return;
-  __threadfence();
-  combine_pair(p, b, h, L, valid);
 }
 
 template <int KB, int VB>
 cudaError_t launch_d(const DecodeArgs& p, cudaStream_t stream) {
   using T = DecodeTraits<KB, VB>;
   static std::atomic<uint64_t> configured{0};   // one bit per device ordinal
+  static int ctas[64] = {};
   int dev = 0;
   cudaError_t e0 = cudaGetDevice(&dev);
   if (e0 != cudaSuccess) return e0;
@@ -775,13 +1042,17 @@ cudaError_t launch_d(const DecodeArgs& p, cudaStream_t stream) {
   if ((configured.load(std::memory_order_acquire) & bit) == 0) {
     cudaError_t e = cudaFuncSetAttribute(decode_kernel<KB, VB>, cudaFuncAttributeMaxDynamicSharedMemorySize, T::kSmem);
     if (e != cudaSuccess) return e;
+    int sms = 0;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    const int n = KVARN_D_MIN_CTAS * sms;
+    ctas[dev & 63] = n < 1 ? 1 : (n > kDecodeMaxCtas ? kDecodeMaxCtas : n);
     configured.fetch_or(bit, std::memory_order_acq_rel);
   }
-  // the per-(seq, KV head) arrival counters start every call at zero
+  // the per-(seq, KV head) unit counters start every call at zero
   cudaError_t e = cudaMemsetAsync(p.counters, 0, static_cast<size_t>(p.B) * p.Hkv * sizeof(int), stream);
   if (e != cudaSuccess) return e;
-  const dim3 grid(static_cast<unsigned>(p.num_splits + 1), static_cast<unsigned>(p.Hkv), static_cast<unsigned>(p.B));
-  decode_kernel<KB, VB><<<grid, kDThreads, T::kSmem, stream>>>(p);
+  decode_kernel<KB, VB><<<ctas[dev & 63], kDThreads, T::kSmem, stream>>>(p);
   return cudaGetLastError();
 }
 
@@ -813,6 +1084,7 @@ cudaError_t noalloc_scratch(void** ptr, size_t* bytes) {
   return cudaSuccess;
 }
 
+// Split-K geometry of the uncompressed baselines (baseline.cu).
 void decode_geometry(int B, int Hkv, int max_blocks, int* tiles_per_split, int* num_splits) {
   // Tiles per split T (a multiple of the 4 warps) chosen to minimise
   // waves x (T / 4 tiles per warp + one tile of fixed cost), with about two
@@ -835,6 +1107,14 @@ void decode_geometry(int B, int Hkv, int max_blocks, int* tiles_per_split, int* 
   if (ns < 1) ns = 1;
   *tiles_per_split = best_t;
   *num_splits = ns;
+}
+
+size_t decode_workspace(int B, int Hq, int Hkv) {
+  const size_t G = Hkv > 0 ? static_cast<size_t>(Hq / Hkv) : 0;
+  const size_t pairs = static_cast<size_t>(B) * Hkv;
+  const size_t records = (pairs + kDecodeMaxCtas) * G + pairs * G;   // tile records, then tail records
+  const size_t counters = (pairs * sizeof(int32_t) + 15) & ~static_cast<size_t>(15);
+  return records * kPartialFloats * sizeof(float) + counters;
 }
 
 cudaError_t launch_decode(const DecodeArgs& p, cudaStream_t stream) {

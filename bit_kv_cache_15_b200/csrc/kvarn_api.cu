@@ -43,7 +43,8 @@ size_t partial_bytes(int B, int Hq, int Hkv, int max_blocks) {
   return static_cast<size_t>(B) * Hq * (ns + 1) * kvarn::kPartialFloats * sizeof(float);
 }
 
-// partial records followed by B * Hkv int32 arrival counters (rounded to 16 bytes)
+// Uncompressed baselines: split-K partial records followed by B * Hkv int32
+// arrival counters (rounded to 16 bytes).
 size_t workspace_for(int B, int Hq, int Hkv, int max_blocks) {
   const size_t counters = (static_cast<size_t>(B) * Hkv * sizeof(int32_t) + 15) & ~static_cast<size_t>(15);
   return partial_bytes(B, Hq, Hkv, max_blocks) + counters;
@@ -125,7 +126,7 @@ size_t kvarn_scale_bytes_per_block(int32_t num_kv_heads) {
 
 size_t kvarn_decode_workspace_bytes(const kvarn_config* cfg, const kvarn_decode_dims* dims) {
   if (kvarn_config_validate(cfg) != KVARN_OK || check_dims(dims, 8) != KVARN_OK) return 0;
-  return workspace_for(dims->num_seqs, dims->num_q_heads, dims->num_kv_heads, dims->max_blocks_per_seq);
+  return kvarn::decode_workspace(dims->num_seqs, dims->num_q_heads, dims->num_kv_heads);
 }
 
 kvarn_status kvarn_quantize_tiles(const void* k, const void* v, const int64_t* slot_mapping, int64_t num_tokens,
@@ -162,7 +163,7 @@ static kvarn_status decode_impl(const void* q, const void* k_new, const void* v_
     return KVARN_ERR_INVALID_ARGUMENT;
   if (append && (k_new == nullptr || v_new == nullptr || !aligned16(k_new) || !aligned16(v_new)))
     return KVARN_ERR_INVALID_ARGUMENT;
-  const size_t need = workspace_for(dims->num_seqs, dims->num_q_heads, dims->num_kv_heads, dims->max_blocks_per_seq);
+  const size_t need = kvarn::decode_workspace(dims->num_seqs, dims->num_q_heads, dims->num_kv_heads);
   if (workspace_bytes < need) return KVARN_ERR_WORKSPACE_TOO_SMALL;
   kvarn::DecodeArgs p;
   p.q = static_cast<const __half*>(q);
@@ -172,10 +173,14 @@ static kvarn_status decode_impl(const void* q, const void* k_new, const void* v_
   p.block_table = block_table;
   p.seq_lens = seq_lens;
   p.out = static_cast<__half*>(out);
-  p.ws = static_cast<float*>(workspace);
-  p.counters = reinterpret_cast<int*>(static_cast<uint8_t*>(workspace) +
-                                      partial_bytes(dims->num_seqs, dims->num_q_heads, dims->num_kv_heads,
-                                                    dims->max_blocks_per_seq));
+  {   // tile records, tail records, counters
+    const size_t pairs = static_cast<size_t>(dims->num_seqs) * dims->num_kv_heads;
+    const size_t G = static_cast<size_t>(dims->num_q_heads / dims->num_kv_heads);
+    float* ws = static_cast<float*>(workspace);
+    p.ws = ws;
+    p.ws_tail = ws + (pairs + kvarn::kDecodeMaxCtas) * G * kvarn::kPartialFloats;
+    p.counters = reinterpret_cast<int*>(p.ws_tail + pairs * G * kvarn::kPartialFloats);
+  }
   p.B = dims->num_seqs;
   p.Hq = dims->num_q_heads;
   p.Hkv = dims->num_kv_heads;
@@ -184,7 +189,6 @@ static kvarn_status decode_impl(const void* q, const void* k_new, const void* v_
   p.num_blocks = dims->num_blocks;
   p.kb = cfg->k_bits;
   p.vb = cfg->v_bits;
-  kvarn::decode_geometry(p.B, p.Hkv, p.max_blocks, &p.tiles_per_split, &p.num_splits);
   p.sm_scale = effective_sm_scale(cfg);
   p.status = dev_status;
   p.append = append;
@@ -225,7 +229,7 @@ kvarn_status kvarn_decode_attention_noalloc(const void* q, const void* packed_ca
   st = check_dims(dims, 8);
   if (st != KVARN_OK) return st;
   if (dims->num_seqs == 0) return KVARN_OK;
-  const size_t need = workspace_for(dims->num_seqs, dims->num_q_heads, dims->num_kv_heads, dims->max_blocks_per_seq);
+  const size_t need = kvarn::decode_workspace(dims->num_seqs, dims->num_q_heads, dims->num_kv_heads);
   if (need > kvarn::kNoAllocScratchBytes) return KVARN_ERR_WORKSPACE_TOO_SMALL;
   void* scratch = nullptr;
   size_t scratch_bytes = 0;

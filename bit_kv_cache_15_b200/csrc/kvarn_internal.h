@@ -35,12 +35,12 @@ struct DecodeArgs {
   const int32_t* block_table;
   const int32_t* seq_lens;
   __half* out;
-  float* ws;            // partial records, then the per-(seq, KV head) counters
-  int* counters;        // B * Hkv arrival counters (zero between calls)
+  float* ws;            // tile partial records [(B * Hkv + kDecodeMaxCtas) * G]
+  float* ws_tail;       // tail partial records [B * Hkv * G]
+  int* counters;        // B * Hkv arrival counters (zeroed by each call)
   int B, Hq, Hkv, G, max_blocks;
   int64_t num_blocks;
   int kb, vb;
-  int tiles_per_split, num_splits;
   float sm_scale;
   int32_t* status;
   // decode step with append (append = 1): seq_lens are the lengths before the
@@ -56,7 +56,14 @@ struct DecodeArgs {
   int iters;
 };
 
-// Split-K geometry: a pure function of the dims (never of seq_lens).
+// Stream-K decode: the work of all (sequence, KV head) pairs -- each pair's
+// full tiles and one tail unit -- is cut into equal contiguous ranges, one per
+// CTA of a grid of two CTAs per SM, at most kDecodeMaxCtas.  The workspace is a
+// function of the dims only (never of seq_lens or the device).
+constexpr int kDecodeMaxCtas = 320;
+size_t decode_workspace(int B, int Hq, int Hkv);
+
+// Split-K geometry of the uncompressed baselines: a pure function of the dims.
 void decode_geometry(int B, int Hkv, int max_blocks, int* tiles_per_split, int* num_splits);
 
 cudaError_t launch_quantize(const QuantArgs& p, cudaStream_t stream);

@@ -104,10 +104,12 @@ KVARN_API size_t kvarn_cache_bytes_per_block(const kvarn_config* cfg, int32_t nu
 /* Bytes of scales per paged block: num_kv_heads * 2 * 528. */
 KVARN_API size_t kvarn_scale_bytes_per_block(int32_t num_kv_heads);
 
-/* Bytes of decode workspace needed for these dims: the split-K partial
- * records followed by one int32 arrival counter per (sequence, KV head).
- * Depends only on cfg and dims (not on seq_lens or the device).  Its
- * contents need no initialisation: each call clears its counters first. */
+/* Bytes of decode workspace needed for these dims: 528-byte partial records
+ * ((B*Hkv + 320) * G for runs of full tiles, B*Hkv*G for the fp16 tails;
+ * 320 bounds the decode grid) followed by one int32 counter per (sequence,
+ * KV head).  Depends only on cfg and dims (not on seq_lens, max_blocks or
+ * the device).  Its contents need no initialisation: each call clears its
+ * counters first. */
 KVARN_API size_t kvarn_decode_workspace_bytes(const kvarn_config* cfg, const kvarn_decode_dims* dims);
 
 /* Quantise-on-write of whole 128-token tiles ([hypho] 四步流水线 steps 1-4;
