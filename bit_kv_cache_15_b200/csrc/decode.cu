@@ -113,14 +113,14 @@ __device__ __forceinline__ float hf(const __half* p, int i) { return __half2floa
 
 // ------------------------------------------------------------------ tail CTA
 
-// Quantise the full fp16 tail tile of (b, h) -- rows 0..126 from the tail
-// buffer, row 127 = the appended token -- into block block_table[b][L / 128]
-// (K then V), by the whole CTA, with the rotation recomputed (no tensor memory).
-// Kept out of line: it runs once per 128 steps of a sequence, and inlined its
-// code pushed the split loop out of the instruction cache (no_instruction
-// stalls 0.2 -> 1.75 per issue, decode 60 -> 66 us under ncu).
+// Quantise one side (K: 0, V: 1) of the full fp16 tail tile of (b, h) --
+// rows 0..126 from the tail buffer, row 127 = the appended token -- into block
+// block_table[b][L / 128], by the whole CTA, with the rotation recomputed (no
+// tensor memory).  Kept out of line: it runs once per 128 steps of a sequence,
+// and inlined its code pushed the split loop out of the instruction cache
+// (no_instruction stalls 0.2 -> 1.75 per issue, decode 60 -> 66 us under ncu).
 template <int KB, int VB>
-__device__ __noinline__ void quantize_full_tail(const DecodeArgs& p, uint8_t* smem, int b, int h, int L) {
+__device__ __noinline__ void quantize_full_tail(const DecodeArgs& p, uint8_t* smem, int b, int h, int L, int side) {
   using namespace qt;
   const int tid = threadIdx.x;
   const int32_t blk = p.block_table[(int64_t)b * p.max_blocks + (L >> 7)];
@@ -130,27 +130,23 @@ __device__ __noinline__ void quantize_full_tail(const DecodeArgs& p, uint8_t* sm
   }
   QuantScratch& sq = *reinterpret_cast<QuantScratch*>(smem + 2 * kBox);
   const uint32_t xs = smem_u32(smem);
-#pragma unroll 1
-  for (int side = 0; side < 2; ++side) {
-    const __half* src = p.tail + (((int64_t)b * 2 + side) * p.Hkv + h) * (int64_t)(kTile * kHeadDim);
-    const __half* nrow = (side == 0 ? p.k_new : p.v_new) + ((int64_t)b * p.Hkv + h) * kHeadDim;
-    // stage row t = tid into the swizzled layout the rotation reads
-    const uint4* row = reinterpret_cast<const uint4*>(tid == kTile - 1 ? nrow : src + (int64_t)tid * kHeadDim);
-#pragma unroll 4
-    for (int c16 = 0; c16 < 16; ++c16) {
-      const uint4 v = __ldg(row + c16);
-      *reinterpret_cast<uint4*>(smem + xoff(tid, c16)) = v;
-    }
-    __syncthreads();
-    TileOut o;
-    o.codes = p.packed_w + ((int64_t)blk * p.Hkv + h) * (int64_t)(2048 * (KB + VB)) + (side == 0 ? 0 : 2048 * KB);
-    o.scales = p.scales_w + (((int64_t)blk * p.Hkv + h) * 2 + side) * (int64_t)kScaleRec;
-    o.dbg = nullptr;
-    o.iters = p.iters;
-    if (side == 0) quantize_tile<0, KB, false>(o, sq, xs, 0u);
-    else quantize_tile<1, VB, false>(o, sq, xs, 0u);
-    __syncthreads();   // the staged tile and the scratch are free again
-  }
+  const __half* src = p.tail + (((int64_t)b * 2 + side) * p.Hkv + h) * (int64_t)(kTile * kHeadDim);
+  const __half* nrow = (side == 0 ? p.k_new : p.v_new) + ((int64_t)b * p.Hkv + h) * kHeadDim;
+  // stage row t = tid into the swizzled layout the rotation reads; all 16
+  // chunks of a row are in flight at once
+  const uint4* row = reinterpret_cast<const uint4*>(tid == kTile - 1 ? nrow : src + (int64_t)tid * kHeadDim);
+#pragma unroll
+  for (int c16 = 0; c16 < 16; ++c16) cp_async16(xs + xoff(tid, c16), row + c16, 16);
+  cp_async_wait_all();
+  __syncthreads();
+  TileOut o;
+  o.codes = p.packed_w + ((int64_t)blk * p.Hkv + h) * (int64_t)(2048 * (KB + VB)) + (side == 0 ? 0 : 2048 * KB);
+  o.scales = p.scales_w + (((int64_t)blk * p.Hkv + h) * 2 + side) * (int64_t)kScaleRec;
+  o.dbg = nullptr;
+  o.iters = p.iters;
+  if (side == 0) quantize_tile<0, KB, false>(o, sq, xs, 0u);
+  else quantize_tile<1, VB, false>(o, sq, xs, 0u);
+  __syncthreads();   // the staged tile and the scratch are free again
 }
 
 // Tail attention (a9) on the tensor cores.  The tail rows (fp16, unrotated)
@@ -166,9 +162,9 @@ __device__ __forceinline__ uint32_t toff(int r, int c16) {
 }
 
 // The tail of (b, h): seq_len % 128 rows, plus the step's own token when
-// appending (taken from k_new / v_new, also written to the tail buffer; a
-// tail it fills is quantised).  Writes one partial record per query head
-// (original domain) to the tail slots.
+// appending (taken from k_new / v_new, and also written to the tail buffer).
+// Writes one partial record per query head (original domain) to the tail
+// slots.
 template <int KB, int VB>
 __device__ void decode_tail(const DecodeArgs& p, uint8_t* smem, int b, int h, int L) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -317,10 +313,6 @@ __device__ void decode_tail(const DecodeArgs& p, uint8_t* smem, int b, int h, in
     __half* vw = p.tail_w + (((int64_t)b * 2 + 1) * p.Hkv + h) * (int64_t)(kTile * kHeadDim) + (int64_t)r * kHeadDim;
     kw[d] = klast[d];
     vw[d] = vlast[d];
-    if (tl == kTile) {
-      __syncthreads();   // the merge area is reused for the staged tile
-      quantize_full_tail<KB, VB>(p, smem, b, h, L);
-    }
   }
 }
 
@@ -761,11 +753,19 @@ __device__ __forceinline__ bool decode_segment(const DecodeArgs& p, uint8_t* sme
 // sequence, so every pair is owned).  The tail, and usually the merge of the
 // pair, fall to the CTA owning the pair's last unit; weighting them as
 // several tiles keeps that CTA's range shorter.
+// A tail that an appended token fills is also quantised, K and V as two more
+// work items of kFillUnits each after the tail (rotation recomputed), so that
+// up to three CTAs share a fill.  Each item falls to the CTA holding its last unit.
 constexpr int kTailUnits = 9;
-__device__ __forceinline__ int pair_units(int L, bool valid) { return (valid ? (L >> 7) : 0) + kTailUnits; }
+constexpr int kFillUnits = 16;
 
 __device__ __forceinline__ bool seq_valid(const DecodeArgs& p, int L) {
   return L >= 0 && L + p.append <= kTile * p.max_blocks;
+}
+__device__ __forceinline__ int pair_tiles(int L, bool valid) { return valid ? (L >> 7) : 0; }
+__device__ __forceinline__ int pair_units(const DecodeArgs& p, int L, bool valid) {
+  const bool fills = valid && p.append && (L & 127) == kTile - 1;
+  return pair_tiles(L, valid) + kTailUnits + (fills ? 2 * kFillUnits : 0);
 }
 
 // CTA i of P owns units [W*i/P, W*(i+1)/P); owner(u) inverts that.
@@ -781,7 +781,7 @@ __device__ void sk_locate(const DecodeArgs& p, int cta, int P, long long* W_out,
   long long mine = 0;
   for (int b = lane; b < p.B; b += 32) {
     const int L = p.seq_lens[b];
-    mine += static_cast<long long>(pair_units(L, seq_valid(p, L))) * p.Hkv;
+    mine += static_cast<long long>(pair_units(p, L, seq_valid(p, L))) * p.Hkv;
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) mine += __shfl_xor_sync(0xffffffffu, mine, o);
@@ -795,7 +795,7 @@ __device__ void sk_locate(const DecodeArgs& p, int cta, int P, long long* W_out,
     long long v = 0;
     if (b < p.B) {
       const int L = p.seq_lens[b];
-      v = static_cast<long long>(pair_units(L, seq_valid(p, L))) * p.Hkv;
+      v = static_cast<long long>(pair_units(p, L, seq_valid(p, L))) * p.Hkv;
     }
     long long incl = v;
 #pragma unroll
@@ -976,12 +976,12 @@ __global__ void __launch_bounds__(kDThreads, KVARN_D_MIN_CTAS) decode_kernel(con
         int b = sh_b;
         long long ps = sh_ps;
         int L = p.seq_lens[b];
-        int nu = pair_units(L, seq_valid(p, L));
+        int nu = pair_units(p, L, seq_valid(p, L));
         if (u >= ps + static_cast<long long>(nu) * p.Hkv) {   // next sequence (each has >= Hkv units)
           ps += static_cast<long long>(nu) * p.Hkv;
           ++b;
           L = p.seq_lens[b];
-          nu = pair_units(L, seq_valid(p, L));
+          nu = pair_units(p, L, seq_valid(p, L));
           sh_b = b;
           sh_ps = ps;
         }
@@ -994,8 +994,18 @@ __global__ void __launch_bounds__(kDThreads, KVARN_D_MIN_CTAS) decode_kernel(con
         sg_nu = nu;
         sg_pst = pst;
         sg_ta = static_cast<int>(u - pst);
-        sg_te = static_cast<int>(min(e - pst, static_cast<long long>(nu - kTailUnits)));
-        sg_tail = e == pst + nu;
+        sg_te = static_cast<int>(min(e - pst, static_cast<long long>(pair_tiles(L, seq_valid(p, L)))));
+        // last units of the work items after the tiles: tail attention, then
+        // (a filling append) quantise K, quantise V
+        const long long m_att = pst + pair_tiles(L, seq_valid(p, L)) + kTailUnits - 1;
+        const int items = nu - pair_tiles(L, seq_valid(p, L)) > kTailUnits ? 3 : 1;
+        int flags = 0;
+#pragma unroll
+        for (int k = 0; k < 3; ++k) {
+          const long long m = m_att + static_cast<long long>(k) * kFillUnits;
+          if (k < items && m >= u && m < e) flags |= 1 << k;
+        }
+        sg_tail = flags;
         sg_done = static_cast<int>(e - u);
         sh_u = e;
       }
@@ -1011,7 +1021,8 @@ __global__ void __launch_bounds__(kDThreads, KVARN_D_MIN_CTAS) decode_kernel(con
       rearm = true;
       woff = (woff + (t_e - t_a) * DecodeTraits<KB, VB>::U) % kDWarps;
     }
-    if (sg_tail) {   // the pair's tail unit
+    const int items = sg_tail;
+    if (items & 1) {   // the pair's tail
       if (!seq_valid(p, L)) {
         if (tid == 0 && h == 0) report_status(p.status, KVARN_DEV_BAD_SEQ_LEN);
       } else {
@@ -1019,13 +1030,16 @@ __global__ void __launch_bounds__(kDThreads, KVARN_D_MIN_CTAS) decode_kernel(con
       }
       __syncthreads();   // shared memory is free again
     }
+#pragma unroll 1
+    for (int side = 0; side < 2; ++side)
+      if (items & (2 << side)) quantize_full_tail<KB, VB>(p, smem, b, h, L, side);
     __threadfence();
     __syncthreads();
     if (tid == 0) sh_last = atomicAdd(p.counters + pair, sg_done) + sg_done == sg_nu;
     __syncthreads();
     if (sh_last) {
       __threadfence();
-      combine_pair(p, b, h, L, seq_valid(p, L), sg_pst, sg_nu - kTailUnits, sh_W, P);
+      combine_pair(p, b, h, L, seq_valid(p, L), sg_pst, pair_tiles(L, seq_valid(p, L)), sh_W, P);
     }
   }
 }
