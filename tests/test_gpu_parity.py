@@ -406,3 +406,21 @@ def test_full_size_qwen3_32b_sampled(K):
     err, bnd, _ = decode_errors(out, ref, heads)
     assert np.all(err <= bnd)
     assert np.all(np.isfinite(out.astype(np.float32)))
+
+
+@pytest.mark.parametrize("lens,hq,hkv,heads", [
+    ([60000 + 77, 5000, 1153, 127, 0], 64, 8, [(0, 0), (0, 37), (1, 8), (2, 63), (3, 5), (4, 0)]),
+    ([40000], 8, 1, [(0, 0), (0, 7)]),
+])
+def test_decode_long_ragged_sampled(K, lens, hq, hkv, heads):
+    """Long, ragged sequences: a pair's tiles span many CTAs of the work split
+    (one 40K sequence alone spreads over every CTA), so the merge walks many
+    records.  Sampled heads against the oracle on the GPU's own cache."""
+    full = sum(L // 128 for L in lens)
+    w = inputs.make_decode_workload("long", lens, hq, hkv, seed=700 + hkv, pool_blocks=full + 3)
+    out, packed_h, scales_h = run_decode(K, w)
+    ref = O.decode(w.q, packed_h, scales_h, w.tail, w.block_table, w.seq_lens, hkv, 4, 2, heads=heads)
+    err, bnd, _ = decode_errors(out, ref, heads)
+    print(f"long ragged Hkv={hkv}: decode max err {err.max():.2e}")
+    assert np.all(err <= bnd)
+    assert np.all(out[[b for b, L in enumerate(lens) if L == 0]] == 0)
