@@ -379,6 +379,7 @@ def precision_sweep(w, dev, iters=30):
                               "bytes": nbytes}
         if (kb, vb) == (4, 2):
             res.update(append_step(w, dev, cfg, kf, vf, slot, q, tail, sl, out, ws, nbytes, timed))
+            res.update(multiquery_step(w, dev, cfg, packed, scales, tail, bt, timed))
         del packed, scales
     # uncompressed caches: full tiles from the same K/V, the tail in one extra block per sequence
     nb = w.num_blocks + BATCH
@@ -408,6 +409,24 @@ def precision_sweep(w, dev, iters=30):
     nbytes = HKV * (n_full_tok + tail_tok) * 256 + 2 * BATCH * HQ * 256
     res["fp8"] = {"us": us, "tokens_per_s": BATCH / (us * 1e-6), "hbm_gbs": nbytes / (us * 1e-6) / 1e9, "bytes": nbytes}
     return res
+
+
+def multiquery_step(w, dev, cfg, packed, scales, tail, bt, timed, q_len=4):
+    """Multi-query attention (a verify step of q_len draft tokens) on the same
+    cache: every sequence's tail holds at least q_len - 1 rows so that all
+    queries sit after its last full tile.  Reports query tokens per second."""
+    import torch
+    from bit_kv_cache_15_b200 import kvarn as K
+    lens = [int(L) // 128 * 128 + max(int(L) % 128, q_len - 1) for L in w.seq_lens]
+    sl = torch.tensor(lens, dtype=torch.int32, device=dev)
+    g = torch.Generator(device=dev).manual_seed(78)
+    q = torch.randn((BATCH, q_len, HQ, 128), generator=g, device=dev).half()
+    out = torch.empty_like(q)
+    d = K.dims(BATCH, HQ, HKV, w.max_blocks_per_seq, w.num_blocks)
+    ws = torch.empty(K.decode_multiquery_workspace_bytes(cfg, d, q_len), dtype=torch.uint8, device=dev)
+    us = timed(lambda: K.decode_attention_multiquery(q, packed, scales, tail, bt, sl, cfg, out=out, workspace=ws))
+    return {f"multiquery{q_len}_k4v2": {"us": us, "query_tokens_per_s": BATCH * q_len / (us * 1e-6),
+                                        "q_len": q_len}}
 
 
 def append_step(w, dev, cfg, kf, vf, slot, q, tail, sl, out, ws, decode_bytes, timed):

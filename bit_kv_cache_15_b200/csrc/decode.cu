@@ -149,6 +149,20 @@ __device__ __noinline__ void quantize_full_tail(const DecodeArgs& p, uint8_t* sm
   __syncthreads();   // the staged tile and the scratch are free again
 }
 
+// Column slot c (0..7) of column group grp of pair (b, h): the columns of a
+// pair are its (query, head) combinations n = i * G + g, 8 per group.  Gives
+// the row of that query head in q / out ([B][qlen][Hq][128]) and the query
+// index; false (and column 0's row, a valid address) past G * qlen.
+__device__ __forceinline__ bool col_row(const DecodeArgs& p, int b, int h, int grp, int c, int64_t* row, int* qi) {
+  const int n = grp * kMaxG + c;
+  const bool live = c < kMaxG && n < p.G * p.qlen;
+  const int nn = live ? n : 0;
+  const int i = nn / p.G, g = nn - (nn / p.G) * p.G;
+  *row = ((int64_t)(b * p.qlen + i) * p.Hq + h * p.G + g) * kHeadDim;
+  *qi = i;
+  return live;
+}
+
 // Tail attention (a9) on the tensor cores.  The tail rows (fp16, unrotated)
 // are staged in 16-row units: K then V, each two 64-channel halves of
 // 16 rows x 128 bytes, 16-byte chunks XOR-swizzled by row so ldmatrix reads
@@ -166,12 +180,12 @@ __device__ __forceinline__ uint32_t toff(int r, int c16) {
 // Writes one partial record per query head (original domain) to the tail
 // slots.
 template <int KB, int VB>
-__device__ void decode_tail(const DecodeArgs& p, uint8_t* smem, int b, int h, int L) {
+__device__ void decode_tail(const DecodeArgs& p, uint8_t* smem, int b, int h, int grp, int L) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g8 = lane >> 2, c = lane & 3;
   const int tl = (L & 127) + p.append;
   if (tl == 0) return;
-  const int G = p.G;
+  const int pw = (b * p.Hkv + h) * p.ngrp + grp;   // work pair: (sequence, KV head, column group)
   const int nun = (tl + kTU - 1) / kTU;
   const __half* kt = p.tail + (((int64_t)b * 2 + 0) * p.Hkv + h) * (int64_t)(kTile * kHeadDim);
   const __half* vt = p.tail + (((int64_t)b * 2 + 1) * p.Hkv + h) * (int64_t)(kTile * kHeadDim);
@@ -191,15 +205,29 @@ __device__ void decode_tail(const DecodeArgs& p, uint8_t* smem, int b, int h, in
     cp_async16(ub + 2 * kTHalf, reinterpret_cast<const uint4*>(vr) + c16, live ? 16 : 0);
   }
   cp_async_wait_all();
-  // q fragments (B operand of q.K): q[g8][16kt + 2c .. +1] and +8; heads >= G are 0
+  // q fragments (B operand of q.K): column g8 at channels 16kt + 2c .. +1 and +8;
+  // columns past G * qlen are 0
   uint32_t qb0[8], qb1[8];
   {
-    const __half* qp = p.q + ((int64_t)b * p.Hq + h * G + (g8 < G ? g8 : 0)) * kHeadDim;
+    int64_t row;
+    int qi;
+    const bool live = col_row(p, b, h, grp, g8, &row, &qi);
+    const __half* qp = p.q + row;
 #pragma unroll
     for (int kt8 = 0; kt8 < 8; ++kt8) {
-      qb0[kt8] = g8 < G ? __ldg(reinterpret_cast<const unsigned int*>(qp + 16 * kt8 + 2 * c)) : 0u;
-      qb1[kt8] = g8 < G ? __ldg(reinterpret_cast<const unsigned int*>(qp + 16 * kt8 + 2 * c + 8)) : 0u;
+      qb0[kt8] = live ? __ldg(reinterpret_cast<const unsigned int*>(qp + 16 * kt8 + 2 * c)) : 0u;
+      qb1[kt8] = live ? __ldg(reinterpret_cast<const unsigned int*>(qp + 16 * kt8 + 2 * c + 8)) : 0u;
     }
+  }
+  // causal limit (last tail row attended) of this lane's columns 2c, 2c + 1:
+  // query i sits at tail row tl - qlen + i (every row for plain decode)
+  int lim[2];
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    int64_t row;
+    int qi;
+    (void)col_row(p, b, h, grp, 2 * c + j, &row, &qi);
+    lim[j] = tl - p.qlen + qi;
   }
   __syncthreads();
 
@@ -224,11 +252,12 @@ __device__ void decode_tail(const DecodeArgs& p, uint8_t* smem, int b, int h, in
       mma_f16(S, a0, a1, a2, a3, qb0[kt8], qb1[kt8]);
     }
     // rows g8 and g8 + 8 (tokens), heads 2c and 2c + 1; tokens past the tail masked
+    const int r0 = un * kTU + g8, r1 = r0 + 8;   // tail rows; causal limits per column
     const bool v0 = g8 < valid_rows, v1 = g8 + 8 < valid_rows;
-    S[0] = v0 ? S[0] * sl : -INFINITY;
-    S[1] = v0 ? S[1] * sl : -INFINITY;
-    S[2] = v1 ? S[2] * sl : -INFINITY;
-    S[3] = v1 ? S[3] * sl : -INFINITY;
+    S[0] = v0 && r0 <= lim[0] ? S[0] * sl : -INFINITY;
+    S[1] = v0 && r0 <= lim[1] ? S[1] * sl : -INFINITY;
+    S[2] = v1 && r1 <= lim[0] ? S[2] * sl : -INFINITY;
+    S[3] = v1 && r1 <= lim[1] ? S[3] * sl : -INFINITY;
     float mx0 = fmaxf(S[0], S[2]), mx1 = fmaxf(S[1], S[3]);
 #pragma unroll
     for (int o = 4; o < 32; o <<= 1) {
@@ -236,11 +265,14 @@ __device__ void decode_tail(const DecodeArgs& p, uint8_t* smem, int b, int h, in
       mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
     }
     const float mn0 = fmaxf(mrun[0], mx0), mn1 = fmaxf(mrun[1], mx1);
-    const float al0 = ex2_fast(mrun[0] - mn0), al1 = ex2_fast(mrun[1] - mn1);
+    // a column with no attended row yet keeps max -inf: exponents are then
+    // taken against 0 so that every weight is 0 instead of NaN
+    const float e0 = mn0 == -INFINITY ? 0.f : mn0, e1 = mn1 == -INFINITY ? 0.f : mn1;
+    const float al0 = ex2_fast(mrun[0] - e0), al1 = ex2_fast(mrun[1] - e1);
     mrun[0] = mn0;
     mrun[1] = mn1;
-    const float p0 = ex2_fast(S[0] - mn0), p1 = ex2_fast(S[1] - mn1);
-    const float p2 = ex2_fast(S[2] - mn0), p3 = ex2_fast(S[3] - mn1);
+    const float p0 = ex2_fast(S[0] - e0), p1 = ex2_fast(S[1] - e1);
+    const float p2 = ex2_fast(S[2] - e0), p3 = ex2_fast(S[3] - e1);
     lsum[0] = lsum[0] * al0 + (p0 + p2);
     lsum[1] = lsum[1] * al1 + (p1 + p3);
     const uint32_t bv0 = movmatrix_t(pack_f2h2(p0, p1));
@@ -286,7 +318,7 @@ __device__ void decode_tail(const DecodeArgs& p, uint8_t* smem, int b, int h, in
     }
   __syncthreads();
   const int d = tid;
-  for (int g = 0; g < G; ++g) {
+  for (int g = 0; g < p.C; ++g) {
     float M = -INFINITY;
 #pragma unroll
     for (int w = 0; w < kDWarps; ++w) M = fmaxf(M, mS[w * kMaxG + g]);
@@ -298,7 +330,7 @@ __device__ void decode_tail(const DecodeArgs& p, uint8_t* smem, int b, int h, in
       l = fmaf(f, lS[w * kMaxG + g], l);
       a = fmaf(f, aS[(w * kMaxG + g) * kHeadDim + d], a);
     }
-    float* rec = p.ws_tail + (((int64_t)b * p.Hkv + h) * G + g) * kPartialFloats;
+    float* rec = p.ws_tail + ((int64_t)pw * p.C + g) * kPartialFloats;
     if (d == 0) {
       rec[0] = M;
       rec[1] = l;
@@ -351,8 +383,8 @@ __device__ __forceinline__ bool issue_unit(const DecodeArgs& p, uint8_t* stage_b
 // the barriers were used by an earlier segment and are invalidated first.
 // Returns false if a copy timed out (the status is set).
 template <int KB, int VB>
-__device__ __forceinline__ bool decode_segment(const DecodeArgs& p, uint8_t* smem, int b, int h, int t_begin,
-                                               int t_end, int woff, bool rearm, float* recs) {
+__device__ __forceinline__ bool decode_segment(const DecodeArgs& p, uint8_t* smem, int b, int h, int grp,
+                                               int t_begin, int t_end, int woff, bool rearm, float* recs) {
   using T = DecodeTraits<KB, VB>;
   constexpr int U = T::U, MT = T::MT;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + T::kBarOff);
@@ -360,7 +392,6 @@ __device__ __forceinline__ bool decode_segment(const DecodeArgs& p, uint8_t* sme
   float* invsig = reinterpret_cast<float*>(smem + T::kInvSigOff);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int G = p.G;
   if (t_begin >= t_end) return true;
 
   if (tid == 0) {
@@ -371,12 +402,14 @@ __device__ __forceinline__ bool decode_segment(const DecodeArgs& p, uint8_t* sme
     fence_barrier_init();
   }
 
-  // ---- q H for the G heads, scaled by a power of two so |q H| <= 1 (a6)
+  // ---- q H for the group's (query, head) columns, scaled by a power of two so |q H| <= 1 (a6)
   {
     const int g = tid >> 4, part = tid & 15;
     float x[8];
-    if (g < G) {
-      const uint4 raw = __ldg(reinterpret_cast<const uint4*>(p.q + ((int64_t)b * p.Hq + h * G + g) * kHeadDim + part * 8));
+    int64_t qrow;
+    int qi;
+    if (col_row(p, b, h, grp, g, &qrow, &qi)) {
+      const uint4 raw = __ldg(reinterpret_cast<const uint4*>(p.q + qrow + part * 8));
       const __half2* hp = reinterpret_cast<const __half2*>(&raw);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -721,7 +754,7 @@ __device__ __forceinline__ bool decode_segment(const DecodeArgs& p, uint8_t* sme
     }
   __syncthreads();
   const int d = tid;
-  for (int g = 0; g < G; ++g) {
+  for (int g = 0; g < p.C; ++g) {
     float M = -INFINITY;
 #pragma unroll
     for (int w = 0; w < kDWarps; ++w) M = fmaxf(M, mS[w * kMaxG + g]);
@@ -759,8 +792,10 @@ __device__ __forceinline__ bool decode_segment(const DecodeArgs& p, uint8_t* sme
 constexpr int kTailUnits = 9;
 constexpr int kFillUnits = 16;
 
+// With qlen > 1 the queries must lie at or after the last full tile's final
+// token ((L mod 128) + 1 >= qlen), so that only the fp16 tail needs causal masks.
 __device__ __forceinline__ bool seq_valid(const DecodeArgs& p, int L) {
-  return L >= 0 && L + p.append <= kTile * p.max_blocks;
+  return L >= 0 && L + p.append <= kTile * p.max_blocks && (p.qlen == 1 || (L >= p.qlen && (L & 127) + 1 >= p.qlen));
 }
 __device__ __forceinline__ int pair_tiles(int L, bool valid) { return valid ? (L >> 7) : 0; }
 __device__ __forceinline__ int pair_units(const DecodeArgs& p, int L, bool valid) {
@@ -781,7 +816,7 @@ __device__ void sk_locate(const DecodeArgs& p, int cta, int P, long long* W_out,
   long long mine = 0;
   for (int b = lane; b < p.B; b += 32) {
     const int L = p.seq_lens[b];
-    mine += static_cast<long long>(pair_units(p, L, seq_valid(p, L))) * p.Hkv;
+    mine += static_cast<long long>(pair_units(p, L, seq_valid(p, L))) * p.Hkv * p.ngrp;
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) mine += __shfl_xor_sync(0xffffffffu, mine, o);
@@ -795,7 +830,7 @@ __device__ void sk_locate(const DecodeArgs& p, int cta, int P, long long* W_out,
     long long v = 0;
     if (b < p.B) {
       const int L = p.seq_lens[b];
-      v = static_cast<long long>(pair_units(p, L, seq_valid(p, L))) * p.Hkv;
+      v = static_cast<long long>(pair_units(p, L, seq_valid(p, L))) * p.Hkv * p.ngrp;
     }
     long long incl = v;
 #pragma unroll
@@ -826,31 +861,33 @@ __device__ void sk_locate(const DecodeArgs& p, int cta, int P, long long* W_out,
 // tail record from its own slot.  One warp per head; lane owns channels
 // 4*lane .. 4*lane + 3.  Records written by other CTAs are read with
 // ld.global.cg (L2), never through L1.
-__device__ void combine_pair(const DecodeArgs& p, int b, int h, int L, bool valid, long long pst, int nt,
+__device__ void combine_pair(const DecodeArgs& p, int b, int h, int grp, int L, bool valid, long long pst, int nt,
                              long long W, int P) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int pair = b * p.Hkv + h;
+  const int pair = (b * p.Hkv + h) * p.ngrp + grp;   // work pair: (sequence, KV head, column group)
   // CTAs whose ranges meet the tiles: owner(pst) .. owner(pst + nt - 1).  With
   // W >= P every CTA range is non-empty, so each of them wrote a record.
   const int i_lo = nt > 0 ? sk_owner(W, P, pst) : 0;
   const int n_rec = nt > 0 ? sk_owner(W, P, pst + nt - 1) - i_lo + 1 : 0;
   const bool dense = W >= P;
   const bool has_tail = (L & 127) + p.append != 0;
-  // a warp merges heads warp and warp + 4 together, so one round of L2 loads
-  // serves both (G <= 8)
+  // a warp merges column slots warp and warp + 4 together, so one round of
+  // L2 loads serves both
   int gh[2];
   bool hl[2];
+  int64_t orow[2];
 #pragma unroll
   for (int k = 0; k < 2; ++k) {
+    int qi;
     gh[k] = warp + kDWarps * k;
-    hl[k] = gh[k] < p.G;
+    hl[k] = col_row(p, b, h, grp, gh[k], &orow[k], &qi);
   }
   if (!hl[0]) return;
   if (!valid || L + p.append == 0) {
 #pragma unroll
     for (int k = 0; k < 2; ++k)
       if (hl[k]) {
-        __half* o = p.out + ((int64_t)b * p.Hq + h * p.G + gh[k]) * kHeadDim + 4 * lane;
+        __half* o = p.out + orow[k] + 4 * lane;
         *reinterpret_cast<uint2*>(o) = make_uint2(0u, 0u);
       }
     return;
@@ -862,7 +899,7 @@ __device__ void combine_pair(const DecodeArgs& p, int b, int h, int L, bool vali
   for (int k = 0; k < 2; ++k) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) a[k][i] = 0.f;
-    const float* trec = p.ws_tail + ((int64_t)pair * p.G + (hl[k] ? gh[k] : 0)) * kPartialFloats;
+    const float* trec = p.ws_tail + ((int64_t)pair * p.C + (hl[k] ? gh[k] : 0)) * kPartialFloats;
     const bool t = has_tail && hl[k];
     mt[k] = t ? __ldcg(trec) : -INFINITY;
     lt[k] = t ? __ldcg(trec + 1) : 0.f;
@@ -880,7 +917,7 @@ __device__ void combine_pair(const DecodeArgs& p, int b, int h, int L, bool vali
 #pragma unroll
       for (int k = 0; k < 2; ++k) {
         const bool lk = live && hl[k];
-        const float* r = p.ws + ((int64_t)(pair + (lk ? i : i_lo)) * p.G + (hl[k] ? gh[k] : 0)) * kPartialFloats;
+        const float* r = p.ws + ((int64_t)(pair + (lk ? i : i_lo)) * p.C + (hl[k] ? gh[k] : 0)) * kPartialFloats;
         mr[k][q] = lk ? __ldcg(r) : -INFINITY;
         lr[k][q] = lk ? __ldcg(r + 1) : 0.f;
         vr[k][q] = lk ? __ldcg(reinterpret_cast<const float4*>(r + 4 + 4 * lane)) : make_float4(0.f, 0.f, 0.f, 0.f);
@@ -932,7 +969,7 @@ __device__ void combine_pair(const DecodeArgs& p, int b, int h, int L, bool vali
     const float il = 1.f / l[k];
     const __half2 o01 = __floats2half2_rn(ak[0] * il, ak[1] * il);
     const __half2 o23 = __floats2half2_rn(ak[2] * il, ak[3] * il);
-    __half* o = p.out + ((int64_t)b * p.Hq + h * p.G + gh[k]) * kHeadDim + 4 * lane;
+    __half* o = p.out + orow[k] + 4 * lane;
     *reinterpret_cast<uint2*>(o) = make_uint2(h2_as_u32(o01), h2_as_u32(o23));
   }
 }
@@ -977,15 +1014,15 @@ __global__ void __launch_bounds__(kDThreads, KVARN_D_MIN_CTAS) decode_kernel(con
         long long ps = sh_ps;
         int L = p.seq_lens[b];
         int nu = pair_units(p, L, seq_valid(p, L));
-        if (u >= ps + static_cast<long long>(nu) * p.Hkv) {   // next sequence (each has >= Hkv units)
-          ps += static_cast<long long>(nu) * p.Hkv;
+        if (u >= ps + static_cast<long long>(nu) * p.Hkv * p.ngrp) {   // next sequence (each has >= Hkv units)
+          ps += static_cast<long long>(nu) * p.Hkv * p.ngrp;
           ++b;
           L = p.seq_lens[b];
           nu = pair_units(p, L, seq_valid(p, L));
           sh_b = b;
           sh_ps = ps;
         }
-        const int h = static_cast<int>((u - ps) / nu);
+        const int h = static_cast<int>((u - ps) / nu);   // sub-pair: KV head x column group
         const long long pst = ps + static_cast<long long>(h) * nu;
         const long long e = min(u_end, pst + nu);
         sg_b = b;
@@ -1013,20 +1050,22 @@ __global__ void __launch_bounds__(kDThreads, KVARN_D_MIN_CTAS) decode_kernel(con
     __syncthreads();
     const int b = sg_b;
     if (b < 0) break;
-    const int h = sg_h, L = sg_L, t_a = sg_ta, t_e = sg_te;
-    const int pair = b * p.Hkv + h;
+    // sub-pair sp of sequence b = (KV head h, column group grp); work pair index
+    const int sp = sg_h, L = sg_L, t_a = sg_ta, t_e = sg_te;
+    const int h = sp / p.ngrp, grp = sp - (sp / p.ngrp) * p.ngrp;
+    const int pair = b * p.Hkv * p.ngrp + sp;
     if (ok && t_a < t_e) {
-      ok = decode_segment<KB, VB>(p, smem, b, h, t_a, t_e, woff, rearm,
-                                  p.ws + static_cast<int64_t>(pair + cta) * p.G * kPartialFloats);
+      ok = decode_segment<KB, VB>(p, smem, b, h, grp, t_a, t_e, woff, rearm,
+                                  p.ws + static_cast<int64_t>(pair + cta) * p.C * kPartialFloats);
       rearm = true;
       woff = (woff + (t_e - t_a) * DecodeTraits<KB, VB>::U) % kDWarps;
     }
     const int items = sg_tail;
     if (items & 1) {   // the pair's tail
       if (!seq_valid(p, L)) {
-        if (tid == 0 && h == 0) report_status(p.status, KVARN_DEV_BAD_SEQ_LEN);
+        if (tid == 0 && sp == 0) report_status(p.status, KVARN_DEV_BAD_SEQ_LEN);
       } else {
-        decode_tail<KB, VB>(p, smem, b, h, L);
+        decode_tail<KB, VB>(p, smem, b, h, grp, L);
       }
       __syncthreads();   // shared memory is free again
     }
@@ -1039,7 +1078,7 @@ __global__ void __launch_bounds__(kDThreads, KVARN_D_MIN_CTAS) decode_kernel(con
     __syncthreads();
     if (sh_last) {
       __threadfence();
-      combine_pair(p, b, h, L, seq_valid(p, L), sg_pst, pair_tiles(L, seq_valid(p, L)), sh_W, P);
+      combine_pair(p, b, h, grp, L, seq_valid(p, L), sg_pst, pair_tiles(L, seq_valid(p, L)), sh_W, P);
     }
   }
 }
@@ -1064,7 +1103,7 @@ cudaError_t launch_d(const DecodeArgs& p, cudaStream_t stream) {
     configured.fetch_or(bit, std::memory_order_acq_rel);
   }
   // the per-(seq, KV head) unit counters start every call at zero
-  cudaError_t e = cudaMemsetAsync(p.counters, 0, static_cast<size_t>(p.B) * p.Hkv * sizeof(int), stream);
+  cudaError_t e = cudaMemsetAsync(p.counters, 0, static_cast<size_t>(p.B) * p.Hkv * p.ngrp * sizeof(int), stream);
   if (e != cudaSuccess) return e;
   decode_kernel<KB, VB><<<ctas[dev & 63], kDThreads, T::kSmem, stream>>>(p);
   return cudaGetLastError();
@@ -1123,10 +1162,13 @@ void decode_geometry(int B, int Hkv, int max_blocks, int* tiles_per_split, int* 
   *num_splits = ns;
 }
 
-size_t decode_workspace(int B, int Hq, int Hkv) {
-  const size_t G = Hkv > 0 ? static_cast<size_t>(Hq / Hkv) : 0;
-  const size_t pairs = static_cast<size_t>(B) * Hkv;
-  const size_t records = (pairs + kDecodeMaxCtas) * G + pairs * G;   // tile records, then tail records
+size_t decode_workspace(int B, int Hq, int Hkv, int qlen) {
+  if (Hkv <= 0 || qlen <= 0) return 0;
+  const size_t cols = static_cast<size_t>(Hq / Hkv) * qlen;              // columns per (sequence, KV head)
+  const size_t ngrp = (cols + kMaxG - 1) / kMaxG;
+  const size_t C = cols < kMaxG ? cols : kMaxG;                           // records per column group
+  const size_t pairs = static_cast<size_t>(B) * Hkv * ngrp;
+  const size_t records = (pairs + kDecodeMaxCtas) * C + pairs * C;       // tile records, then tail records
   const size_t counters = (pairs * sizeof(int32_t) + 15) & ~static_cast<size_t>(15);
   return records * kPartialFloats * sizeof(float) + counters;
 }

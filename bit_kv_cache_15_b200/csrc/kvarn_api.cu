@@ -126,7 +126,7 @@ size_t kvarn_scale_bytes_per_block(int32_t num_kv_heads) {
 
 size_t kvarn_decode_workspace_bytes(const kvarn_config* cfg, const kvarn_decode_dims* dims) {
   if (kvarn_config_validate(cfg) != KVARN_OK || check_dims(dims, 8) != KVARN_OK) return 0;
-  return kvarn::decode_workspace(dims->num_seqs, dims->num_q_heads, dims->num_kv_heads);
+  return kvarn::decode_workspace(dims->num_seqs, dims->num_q_heads, dims->num_kv_heads, 1);
 }
 
 kvarn_status kvarn_quantize_tiles(const void* k, const void* v, const int64_t* slot_mapping, int64_t num_tokens,
@@ -149,7 +149,7 @@ static kvarn_status decode_impl(const void* q, const void* k_new, const void* v_
                                 const void* scales, const void* fp16_tail, const int32_t* block_table,
                                 const int32_t* seq_lens, void* out, const kvarn_decode_dims* dims,
                                 const kvarn_config* cfg, void* workspace, size_t workspace_bytes, int32_t* dev_status,
-                                void* stream, int append) {
+                                void* stream, int append, int32_t q_len) {
   kvarn_status st = kvarn_config_validate(cfg);
   if (st != KVARN_OK) return st;
   st = check_dims(dims, 8);
@@ -163,7 +163,8 @@ static kvarn_status decode_impl(const void* q, const void* k_new, const void* v_
     return KVARN_ERR_INVALID_ARGUMENT;
   if (append && (k_new == nullptr || v_new == nullptr || !aligned16(k_new) || !aligned16(v_new)))
     return KVARN_ERR_INVALID_ARGUMENT;
-  const size_t need = kvarn::decode_workspace(dims->num_seqs, dims->num_q_heads, dims->num_kv_heads);
+  if (q_len < 1 || q_len > KVARN_MAX_Q_LEN || (append && q_len != 1)) return KVARN_ERR_INVALID_ARGUMENT;
+  const size_t need = kvarn::decode_workspace(dims->num_seqs, dims->num_q_heads, dims->num_kv_heads, q_len);
   if (workspace_bytes < need) return KVARN_ERR_WORKSPACE_TOO_SMALL;
   kvarn::DecodeArgs p;
   p.q = static_cast<const __half*>(q);
@@ -173,13 +174,17 @@ static kvarn_status decode_impl(const void* q, const void* k_new, const void* v_
   p.block_table = block_table;
   p.seq_lens = seq_lens;
   p.out = static_cast<__half*>(out);
-  {   // tile records, tail records, counters
-    const size_t pairs = static_cast<size_t>(dims->num_seqs) * dims->num_kv_heads;
-    const size_t G = static_cast<size_t>(dims->num_q_heads / dims->num_kv_heads);
+  {   // tile records, tail records, counters; per (sequence, KV head) the
+      // G * q_len (query, head) columns form groups of up to 8
+    const int cols = (dims->num_q_heads / dims->num_kv_heads) * q_len;
+    p.qlen = q_len;
+    p.ngrp = (cols + 7) / 8;
+    p.C = cols < 8 ? cols : 8;
+    const size_t pairs = static_cast<size_t>(dims->num_seqs) * dims->num_kv_heads * p.ngrp;
     float* ws = static_cast<float*>(workspace);
     p.ws = ws;
-    p.ws_tail = ws + (pairs + kvarn::kDecodeMaxCtas) * G * kvarn::kPartialFloats;
-    p.counters = reinterpret_cast<int*>(p.ws_tail + pairs * G * kvarn::kPartialFloats);
+    p.ws_tail = ws + (pairs + kvarn::kDecodeMaxCtas) * p.C * kvarn::kPartialFloats;
+    p.counters = reinterpret_cast<int*>(p.ws_tail + pairs * p.C * kvarn::kPartialFloats);
   }
   p.B = dims->num_seqs;
   p.Hq = dims->num_q_heads;
@@ -206,7 +211,23 @@ kvarn_status kvarn_decode_attention(const void* q, const void* packed_cache, con
                                     void* out, const kvarn_decode_dims* dims, const kvarn_config* cfg,
                                     void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream) {
   return decode_impl(q, nullptr, nullptr, packed_cache, scales, fp16_tail, block_table, seq_lens, out, dims, cfg,
-                     workspace, workspace_bytes, dev_status, stream, 0);
+                     workspace, workspace_bytes, dev_status, stream, 0, 1);
+}
+
+size_t kvarn_decode_multiquery_workspace_bytes(const kvarn_config* cfg, const kvarn_decode_dims* dims,
+                                               int32_t q_len) {
+  if (kvarn_config_validate(cfg) != KVARN_OK || check_dims(dims, 8) != KVARN_OK) return 0;
+  if (q_len < 1 || q_len > KVARN_MAX_Q_LEN) return 0;
+  return kvarn::decode_workspace(dims->num_seqs, dims->num_q_heads, dims->num_kv_heads, q_len);
+}
+
+kvarn_status kvarn_decode_attention_multiquery(const void* q, int32_t q_len, const void* packed_cache,
+                                               const void* scales, const void* fp16_tail, const int32_t* block_table,
+                                               const int32_t* seq_lens, void* out, const kvarn_decode_dims* dims,
+                                               const kvarn_config* cfg, void* workspace, size_t workspace_bytes,
+                                               int32_t* dev_status, void* stream) {
+  return decode_impl(q, nullptr, nullptr, packed_cache, scales, fp16_tail, block_table, seq_lens, out, dims, cfg,
+                     workspace, workspace_bytes, dev_status, stream, 0, q_len);
 }
 
 kvarn_status kvarn_decode_attention_append(const void* q, const void* k_new, const void* v_new, void* packed_cache,
@@ -215,7 +236,7 @@ kvarn_status kvarn_decode_attention_append(const void* q, const void* k_new, con
                                            const kvarn_config* cfg, void* workspace, size_t workspace_bytes,
                                            int32_t* dev_status, void* stream) {
   return decode_impl(q, k_new, v_new, packed_cache, scales, fp16_tail, block_table, seq_lens, out, dims, cfg,
-                     workspace, workspace_bytes, dev_status, stream, 1);
+                     workspace, workspace_bytes, dev_status, stream, 1, 1);
 }
 
 kvarn_status kvarn_decode_attention_noalloc(const void* q, const void* packed_cache, const void* scales,
@@ -229,7 +250,7 @@ kvarn_status kvarn_decode_attention_noalloc(const void* q, const void* packed_ca
   st = check_dims(dims, 8);
   if (st != KVARN_OK) return st;
   if (dims->num_seqs == 0) return KVARN_OK;
-  const size_t need = kvarn::decode_workspace(dims->num_seqs, dims->num_q_heads, dims->num_kv_heads);
+  const size_t need = kvarn::decode_workspace(dims->num_seqs, dims->num_q_heads, dims->num_kv_heads, 1);
   if (need > kvarn::kNoAllocScratchBytes) return KVARN_ERR_WORKSPACE_TOO_SMALL;
   void* scratch = nullptr;
   size_t scratch_bytes = 0;

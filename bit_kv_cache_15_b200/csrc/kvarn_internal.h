@@ -47,6 +47,11 @@ struct DecodeArgs {
   // step; each (seq, KV head) first takes k_new / v_new ([B][Hkv][128]) as its
   // token at position seq_len, written to the fp16 tail; a tail that this
   // fills (128 tokens) is quantised into block block_table[seq][seq_len / 128]
+  // multi-query (qlen > 1): q and out are [B][qlen][Hq][128]; query i of
+  // sequence b sits at position seq_len - qlen + i and attends keys up to it.
+  // A (sequence, KV head) pair's G * qlen columns (query, head) are processed
+  // in ngrp groups of up to 8; C = min(8, G * qlen) records per group.
+  int qlen, ngrp, C;
   int append;
   const __half* k_new;
   const __half* v_new;
@@ -61,7 +66,7 @@ struct DecodeArgs {
 // CTA of a grid of two CTAs per SM, at most kDecodeMaxCtas.  The workspace is a
 // function of the dims only (never of seq_lens or the device).
 constexpr int kDecodeMaxCtas = 320;
-size_t decode_workspace(int B, int Hq, int Hkv);
+size_t decode_workspace(int B, int Hq, int Hkv, int qlen);
 
 // Split-K geometry of the uncompressed baselines: a pure function of the dims.
 void decode_geometry(int B, int Hkv, int max_blocks, int* tiles_per_split, int* num_splits);

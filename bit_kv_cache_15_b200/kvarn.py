@@ -65,6 +65,9 @@ _SIGS = {
                                              ctypes.POINTER(Config), _vp, _vp]),
     "kvarn_decode_attention_append": (_st, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(DecodeDims),
                                             ctypes.POINTER(Config), _vp, _sz, _vp, _vp]),
+    "kvarn_decode_multiquery_workspace_bytes": (_sz, [ctypes.POINTER(Config), ctypes.POINTER(DecodeDims), _i32]),
+    "kvarn_decode_attention_multiquery": (_st, [_vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(DecodeDims),
+                                                ctypes.POINTER(Config), _vp, _sz, _vp, _vp]),
     "kvarn_baseline_workspace_bytes": (_sz, [ctypes.POINTER(DecodeDims)]),
     "kvarn_decode_attention_fp16": (_st, [_vp, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(DecodeDims),
                                           ctypes.c_float, _vp, _sz, _vp, _vp]),
@@ -234,6 +237,41 @@ def decode_attention_append(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.T
                                             workspace.numel() * workspace.element_size(), _ptr(dev_status),
                                             _stream(stream))
     _check("kvarn_decode_attention_append", st)
+    return out
+
+
+def decode_multiquery_workspace_bytes(cfg: Config, d: DecodeDims, q_len: int) -> int:
+    return int(_lib.kvarn_decode_multiquery_workspace_bytes(ctypes.byref(cfg), ctypes.byref(d), int(q_len)))
+
+
+def decode_attention_multiquery(q: torch.Tensor, packed_cache: torch.Tensor, scales: torch.Tensor,
+                                fp16_tail: torch.Tensor, block_table: torch.Tensor, seq_lens: torch.Tensor,
+                                cfg: Config, out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                                dev_status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Multi-query attention over the packed cache (kvarn_decode_attention_multiquery
+    in include/kvarn.h): q [B][q_len][Hq][128] fp16, query i of sequence b at
+    position seq_len - q_len + i, attending causally.  Returns out like q."""
+    _need(q, "q", torch.float16)
+    _need(packed_cache, "packed_cache", torch.uint8)
+    _need(scales, "scales", torch.uint8)
+    _need(fp16_tail, "fp16_tail", torch.float16)
+    _need(block_table, "block_table", torch.int32)
+    _need(seq_lens, "seq_lens", torch.int32)
+    if q.dim() != 4:
+        raise ValueError("q must be [B][q_len][Hq][128]")
+    B, q_len, Hq, _ = q.shape
+    Hkv = int(packed_cache.shape[1])
+    d = dims(B, Hq, Hkv, int(block_table.shape[1]), int(packed_cache.shape[0]))
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = torch.zeros(decode_multiquery_workspace_bytes(cfg, d, q_len), dtype=torch.uint8, device=q.device)
+    st = _lib.kvarn_decode_attention_multiquery(_ptr(q), int(q_len), _ptr(packed_cache), _ptr(scales),
+                                                _ptr(fp16_tail), _ptr(block_table), _ptr(seq_lens), _ptr(out),
+                                                ctypes.byref(d), ctypes.byref(cfg), _ptr(workspace),
+                                                workspace.numel() * workspace.element_size(), _ptr(dev_status),
+                                                _stream(stream))
+    _check("kvarn_decode_attention_multiquery", st)
     return out
 
 

@@ -50,6 +50,7 @@ extern "C" {
 #define KVARN_ABI_VERSION 1
 #define KVARN_TILE_TOKENS 128
 #define KVARN_HEAD_DIM 128
+#define KVARN_MAX_Q_LEN 128   /* queries per sequence of kvarn_decode_attention_multiquery */
 /* bytes of one scale record (per block, KV head and K-or-V):
  * fp16 lt[128] | fp16 lc[128] | fp32 zero | fp32 step | 8 B pad */
 #define KVARN_SCALE_RECORD_BYTES 528
@@ -199,6 +200,34 @@ KVARN_API kvarn_status kvarn_decode_attention_append(const void* q, const void* 
                                                      const kvarn_decode_dims* dims, const kvarn_config* cfg,
                                                      void* workspace, size_t workspace_bytes,
                                                      int32_t* dev_status, void* stream);
+
+/* Multi-query attention over the packed cache: q_len query tokens per
+ * sequence, each attending causally -- the shape of a speculative-decoding
+ * verify step or a short chunk of chunked prefill.  The pages quote
+ * time-to-first-token figures but give no kernel for it; this is the decode
+ * path with (query, head) columns in place of heads.
+ *
+ *  q      fp16 [B][q_len][Hq][128]: query i of sequence b sits at position
+ *         seq_len - q_len + i and attends keys [0, seq_len - q_len + i].
+ *  out    fp16 [B][q_len][Hq][128].
+ *  The q_len tokens' own K/V must already be in the cache (normally in the
+ *  fp16 tail, e.g. by kvarn_decode_attention_append); seq_len counts them.
+ *  Other arguments as kvarn_decode_attention.
+ *  workspace  at least kvarn_decode_multiquery_workspace_bytes(cfg, dims, q_len).
+ * Requires 1 <= q_len <= KVARN_MAX_Q_LEN.  Every query must lie at or after the
+ * final token of the last full tile, i.e. (seq_len mod 128) + 1 >= q_len and
+ * seq_len >= q_len: then only the fp16 tail is masked.  A sequence that breaks
+ * this is reported as KVARN_DEV_BAD_SEQ_LEN and its outputs are 0.  q_len = 1
+ * is exactly kvarn_decode_attention. */
+KVARN_API size_t kvarn_decode_multiquery_workspace_bytes(const kvarn_config* cfg, const kvarn_decode_dims* dims,
+                                                         int32_t q_len);
+
+KVARN_API kvarn_status kvarn_decode_attention_multiquery(const void* q, int32_t q_len, const void* packed_cache,
+                                                         const void* scales, const void* fp16_tail,
+                                                         const int32_t* block_table, const int32_t* seq_lens,
+                                                         void* out, const kvarn_decode_dims* dims,
+                                                         const kvarn_config* cfg, void* workspace,
+                                                         size_t workspace_bytes, int32_t* dev_status, void* stream);
 
 /* Size of the fixed device scratch used by kvarn_decode_attention_noalloc. */
 #define KVARN_NOALLOC_SCRATCH_BYTES (8u << 20)

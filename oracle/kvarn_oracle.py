@@ -397,6 +397,35 @@ def decode_append(q, k_new, v_new, packed, scales, tail, block_table, seq_lens, 
     return out, packed2, scales2, tail2
 
 
+def decode_multiquery(q, packed, scales, tail, block_table, seq_lens, num_kv_heads: int, kb: int, vb: int,
+                      sm_scale: float | None = None, heads=None) -> np.ndarray:
+    """Multi-query attention over the cache, causal.
+
+    Reading (the pages quote time-to-first-token but fix no multi-query
+    kernel): q is [B][qlen][Hq][128] fp16; query i of sequence b sits at
+    position L - qlen + i (L = seq_lens[b], counting the queries' own tokens)
+    and attends keys [0, L - qlen + i], read as decode reads them.  Defined
+    when L >= qlen and (L % 128) + 1 >= qlen (every query at or after the last
+    full tile's final token); other sequences, and empty ones, give 0.
+    `heads`: optional (b, i, j) triples to compute.  Returns [B][qlen][Hq][128] fp16.
+    """
+    B, qlen, Hq, _ = q.shape
+    G = Hq // num_kv_heads
+    if sm_scale is None:
+        sm_scale = 1.0 / np.sqrt(HEAD_DIM)
+    out = np.zeros((B, qlen, Hq, HEAD_DIM), dtype=np.float16)
+    trip = heads if heads is not None else [(b, i, j) for b in range(B) for i in range(qlen) for j in range(Hq)]
+    cache = {}
+    for b, i, j in trip:
+        L = int(seq_lens[b])
+        if L < qlen or (L % TILE) + 1 < qlen or L == 0:
+            continue
+        K, V = gather_kv(packed, scales, tail, block_table, L, b, j // G, kb, vb, cache)
+        lim = L - qlen + i + 1
+        out[b, i, j] = attention(q[b, i, j], K[:lim], V[:lim], sm_scale).astype(np.float16)
+    return out
+
+
 def decode_folded(q, packed, scales, tail, block_table, seq_lens, num_kv_heads: int, kb: int, vb: int,
                   sm_scale: float | None = None, heads=None) -> np.ndarray:
     """The same attention with every scale folded in on read, fp64 (returns

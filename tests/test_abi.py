@@ -138,3 +138,20 @@ def test_decode_append_argument_checks():
     assert call(v_new=FAKE + 4) == 1                   # misaligned
     assert call(ws_bytes=need - 1) == 4
     assert call(dd=K.dims(0, 8, 2, 4, 16)) == 0         # empty batch: nothing to do
+
+
+def test_multiquery_argument_checks():
+    cfg = K.config()
+    d = K.dims(2, 8, 2, 4, 16)
+    need = K.decode_multiquery_workspace_bytes(cfg, d, 4)
+    assert need > K.decode_workspace_bytes(cfg, d)           # 16 columns per KV head: two groups
+    assert K.decode_multiquery_workspace_bytes(cfg, d, 1) == K.decode_workspace_bytes(cfg, d)
+    assert K.decode_multiquery_workspace_bytes(cfg, d, 0) == 0
+
+    def call(q_len, ws_bytes=need):
+        return K.lib.kvarn_decode_attention_multiquery(FAKE, q_len, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                                       ctypes.byref(d), ctypes.byref(cfg), FAKE, ws_bytes, None, None)
+
+    assert call(0) == 1
+    assert call(129) == 1
+    assert call(4, need - 1) == 4

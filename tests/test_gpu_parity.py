@@ -424,3 +424,34 @@ def test_decode_long_ragged_sampled(K, lens, hq, hkv, heads):
     print(f"long ragged Hkv={hkv}: decode max err {err.max():.2e}")
     assert np.all(err <= bnd)
     assert np.all(out[[b for b, L in enumerate(lens) if L == 0]] == 0)
+
+
+# ------------------------------------------------------------------ multi-query
+
+@pytest.mark.parametrize("hq,hkv,qlen", [(64, 8, 4), (8, 8, 3), (16, 2, 2), (8, 2, 1)])
+def test_decode_multiquery_parity(K, hq, hkv, qlen):
+    """q_len queries per sequence, causal: (query, head) columns in groups of
+    8 per KV head (4 groups at 64/8 heads x 4 queries).  Lengths cover a query
+    block ending a full tile, a tail-only sequence, long sequences and one
+    that breaks the precondition (tail shorter than q_len - 1)."""
+    lens = [256 + qlen - 1, 1024 + 127, 40 * 128 + 10, 7 + qlen, 128 + max(qlen - 2, 0), 3 * 128 + 50]
+    full = sum(L // 128 for L in lens)
+    w = inputs.make_decode_workload("mq", lens, hq, hkv, seed=800 + qlen, pool_blocks=full + 2)
+    cfg = K.config()
+    packed, scales = K.alloc_cache(cfg, w.num_blocks, hkv)
+    K.quantize_tiles(_dev(w.k_full), _dev(w.v_full), _dev(w.slot_mapping), packed, scales, cfg)
+    q = np.random.default_rng(801).standard_normal((len(lens), qlen, hq, 128)).astype(np.float16)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = K.decode_attention_multiquery(_dev(q), packed, scales, _dev(w.tail), _dev(w.block_table), _dev(w.seq_lens),
+                                        cfg, dev_status=status).cpu().numpy()
+    torch.cuda.synchronize()
+    bad = [b for b, L in enumerate(lens) if not (L >= qlen and L % 128 + 1 >= qlen)]
+    assert int(status.item()) == (3 if bad else 0)
+    ref = O.decode_multiquery(q, packed.cpu().numpy(), scales.cpu().numpy(), w.tail, w.block_table, w.seq_lens,
+                              hkv, 4, 2)
+    err = np.abs(out.astype(np.float64) - ref.astype(np.float64))
+    bnd = decode_bound(ref)
+    print(f"multiquery {hq}/{hkv} q_len={qlen}: max err {err.max():.2e}")
+    assert np.all(err <= bnd)
+    for b in bad:
+        assert np.all(out[b] == 0)

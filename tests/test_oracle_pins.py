@@ -438,3 +438,32 @@ def test_append_fill_quantises_the_tile_like_the_write_path():
     k, v = _rows_after_append(w, k_new, v_new, b)
     ref = O.decode_uncompressed(w.q[b:b + 1], [k], [v], np.array([128]), 2)
     assert np.array_equal(out[b], ref[0])
+
+
+# ---------------------------------------------------------------------------
+# multi-query attention
+# ---------------------------------------------------------------------------
+
+def test_multiquery_single_query_is_decode():
+    w = inputs.make_decode_workload("mq", [300, 129, 0, 128], 8, 2, seed=61, pool_blocks=8)
+    packed, scales = O.quantize_tiles(w.k_full, w.v_full, w.slot_mapping, 2, w.num_blocks, 4, 2)
+    out = O.decode_multiquery(w.q[:, None], packed, scales, w.tail, w.block_table, w.seq_lens, 2, 4, 2)
+    ref = O.decode(w.q, packed, scales, w.tail, w.block_table, w.seq_lens, 2, 4, 2)
+    assert np.array_equal(out[:, 0], ref)
+
+
+def test_multiquery_query_i_is_decode_of_the_prefix_it_sees():
+    """Query i attends exactly the first L - qlen + i + 1 tokens: the plain
+    decode of a sequence cut to that length, over the same cache."""
+    qlen = 5
+    lens = [256 + 4, 128 + 100, 20, 128 + 3]          # the last one breaks the precondition (3 + 1 < 5)
+    w = inputs.make_decode_workload("mq", lens, 8, 2, seed=63, pool_blocks=8)
+    packed, scales = O.quantize_tiles(w.k_full, w.v_full, w.slot_mapping, 2, w.num_blocks, 4, 2)
+    q = np.random.default_rng(64).standard_normal((len(lens), qlen, 8, 128)).astype(np.float16)
+    out = O.decode_multiquery(q, packed, scales, w.tail, w.block_table, w.seq_lens, 2, 4, 2)
+    for i in range(qlen):
+        cut = np.array([L - qlen + i + 1 for L in lens], dtype=np.int32)
+        ref = O.decode(q[:, i], packed, scales, w.tail, w.block_table, cut, 2, 4, 2)
+        for b in range(3):
+            assert np.array_equal(out[b, i], ref[b])
+    assert np.all(out[3] == 0)
