@@ -1,10 +1,11 @@
-"""Data-parallel sharding of the hot path over ranks (one process per GPU).
+"""Sharding of the hot path over ranks (one process per GPU).
 
 The path splits into independent units -- quantisation tiles and decode
-(sequence, KV head) problems -- with no exchange step between them, so N
-GPUs each take their own sequences and never communicate on the data path.
-Only the benchmark's timing uses a collective (the max of the per-rank
-elapsed times).
+(sequence, KV head) problems -- with no exchange step between them.  N GPUs
+either take their own sequences (data parallel) or their own KV heads with
+the query heads that read them (tensor parallel over heads, the pages' TP
+setting), and never communicate on the data path.  Only the benchmark's
+timing uses a collective (the max of the per-rank elapsed times).
 """
 from __future__ import annotations
 
@@ -16,6 +17,17 @@ def shard_range(global_units: int, rank: int, world: int) -> tuple[int, int]:
     base, extra = divmod(global_units, world)
     start = rank * base + min(rank, extra)
     return start, start + base + (1 if rank < extra else 0)
+
+
+def kv_head_shard(num_kv_heads: int, num_q_heads: int, rank: int, world: int) -> tuple[range, range]:
+    """KV heads of `rank` and the query heads that read them.  Query head j
+    reads KV head j // (Hq / Hkv), so a contiguous block of KV heads owns the
+    matching contiguous block of query heads; world must divide Hkv."""
+    if world <= 0 or not 0 <= rank < world or num_kv_heads % world or num_q_heads % num_kv_heads:
+        raise ValueError("KV heads must split evenly over the ranks")
+    per = num_kv_heads // world
+    g = num_q_heads // num_kv_heads
+    return range(rank * per, (rank + 1) * per), range(rank * per * g, (rank + 1) * per * g)
 
 
 def rank_seed(seed: int, rank: int) -> int:
