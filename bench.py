@@ -132,17 +132,24 @@ def algorithmic_bytes(w, n_append_tokens):
     return q_bytes, d_bytes
 
 
+def source_sha(files):
+    """Hash of a kernel's source files (the .cu and the headers it includes)."""
+    h = hashlib.sha256()
+    for f in files:
+        h.update(open(os.path.join(ROOT, "bit_kv_cache_15_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
 def traffic_record(kernel):
-    """DRAM bytes per launch from a committed ncu capture, if the kernel source is unchanged since."""
+    """DRAM bytes per launch from a committed ncu capture, if the kernel's
+    sources are unchanged since."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     rec = json.load(open(p)).get(kernel)
     if not rec:
         return None
-    src = os.path.join(ROOT, "bit_kv_cache_15_b200", "csrc", rec["source"])
-    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    return rec["bytes_per_launch"] if sha == rec["source_sha"] else None
+    return rec["bytes_per_launch"] if source_sha(rec["sources"]) == rec["sources_sha"] else None
 
 
 # ------------------------------------------------------------------ our arm
