@@ -455,3 +455,32 @@ def test_decode_multiquery_parity(K, hq, hkv, qlen):
     assert np.all(err <= bnd)
     for b in bad:
         assert np.all(out[b] == 0)
+
+
+def test_decode_many_short_sequences(K):
+    """100 ragged sequences (0 to 600 tokens): the work split's start search
+    scans the sequences 32 at a time, and most CTAs straddle several pairs."""
+    rng = np.random.default_rng(900)
+    lens = [int(x) for x in rng.integers(0, 600, size=100)]
+    lens[7] = 0
+    full = sum(L // 128 for L in lens)
+    w = inputs.make_decode_workload("many", lens, 4, 2, seed=901, pool_blocks=full + 1)
+    out, packed_h, scales_h = run_decode(K, w)
+    heads = [(b, j) for b in range(0, 100, 3) for j in (0, 3)]
+    ref = O.decode(w.q, packed_h, scales_h, w.tail, w.block_table, w.seq_lens, 2, 4, 2, heads=heads)
+    err, bnd, _ = decode_errors(out, ref, heads)
+    assert np.all(err <= bnd)
+    assert np.all(out[7] == 0)
+    # the same cache read as 3-query verify steps (sequences with < 2 tail rows give 0)
+    cfg = K.config()
+    q = rng.standard_normal((100, 3, 4, 128)).astype(np.float16)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    mq = K.decode_attention_multiquery(_dev(q), torch.from_numpy(packed_h).cuda(), torch.from_numpy(scales_h).cuda(),
+                                       _dev(w.tail), _dev(w.block_table), _dev(w.seq_lens), cfg,
+                                       dev_status=status).cpu().numpy()
+    torch.cuda.synchronize()
+    trip = [(b, i, j) for b in range(1, 100, 4) for i in range(3) for j in (1, 2)]
+    ref3 = O.decode_multiquery(q, packed_h, scales_h, w.tail, w.block_table, w.seq_lens, 2, 4, 2, heads=trip)
+    for b, i, j in trip:
+        e = np.abs(mq[b, i, j].astype(np.float64) - ref3[b, i, j].astype(np.float64))
+        assert np.all(e <= decode_bound(ref3[b, i, j])), (b, i, j)
