@@ -54,6 +54,15 @@ __device__ __forceinline__ float lg2_approx(float x) {
   return y;
 }
 
+// The weight 2^(-2 l) of a log-scale l = log2_scale(sum): 128 / sum, with the
+// same floor.  Used inside the passes, where only the weights are needed; the
+// stored log-scales come from log2_scale of the last pass's sums.
+__device__ __forceinline__ float weight_of_sum(float sum_sq) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;\n" : "=f"(r) : "f"(fmaxf(sum_sq, 4.547473508864641e-13f)));
+  return 128.f * r;
+}
+
 // 1/2 log2 of the mean square (sum / 128), floored at 2^-48
 __device__ __forceinline__ float log2_scale(float sum_sq) {
   return 0.5f * (lg2_approx(fmaxf(sum_sq, 4.547473508864641e-13f)) - 7.0f);   // 2^-41
@@ -88,11 +97,22 @@ __device__ __forceinline__ void fwht8x2(float2 (&v)[8]) {
 template <int N>
 __device__ __forceinline__ void rs_step(float* v, int mask, int lane) {
   const bool up = (lane & mask) != 0;
+  float keep[N / 2], recv[N / 2];
 #pragma unroll
   for (int i = 0; i < N / 2; ++i) {
     const float send = up ? v[i] : v[i + N / 2];
-    const float keep = up ? v[i + N / 2] : v[i];
-    v[i] = keep + __shfl_xor_sync(0xffffffffu, send, mask);
+    keep[i] = up ? v[i + N / 2] : v[i];
+    recv[i] = __shfl_xor_sync(0xffffffffu, send, mask);
+  }
+  if constexpr (N / 2 >= 2) {   // the adds in f32x2 pairs
+#pragma unroll
+    for (int i = 0; i < N / 2; i += 2) {
+      const float2 r = __fadd2_rn(make_float2(keep[i], keep[i + 1]), make_float2(recv[i], recv[i + 1]));
+      v[i] = r.x;
+      v[i + 1] = r.y;
+    }
+  } else {
+    v[0] = keep[0] + recv[0];
   }
 }
 
@@ -286,7 +306,7 @@ __device__ __forceinline__ void quantize_tile(const TileOut& o, QuantScratch& sm
   float wt[NT];                           // token weights 2^(-2 lt)
 #pragma unroll
   for (int i = 0; i < NT; ++i) wt[i] = 1.f;
-  float lt_own = 0.f, lc_own = 0.f;
+  float lt_sum = 1.f, lc_sum = 1.f;   // this thread's token / channel sums of the last pass
 
   for (int it = 0; it < o.iters; ++it) {
     // channel pass: partial sums over this thread's tokens
@@ -338,8 +358,8 @@ __device__ __forceinline__ void quantize_tile(const TileOut& o, QuantScratch& sm
     __syncthreads();
     {
       const float tot = (sm.red[0][tid] + sm.red[1][tid]) + (sm.red[2][tid] + sm.red[3][tid]);
-      lc_own = log2_scale(tot);
-      sm.u[tid] = ex2_fast(-2.f * lc_own);
+      lc_sum = tot;
+      sm.u[tid] = weight_of_sum(tot);
     }
     __syncthreads();
 
@@ -370,8 +390,8 @@ __device__ __forceinline__ void quantize_tile(const TileOut& o, QuantScratch& sm
         }
       rs_step<4>(s, 2, lane);
       rs_step<2>(s, 1, lane);
-      lt_own = log2_scale(s[0]);
-      const float wown = ex2_fast(-2.f * lt_own);
+      lt_sum = s[0];
+      const float wown = weight_of_sum(s[0]);
 #pragma unroll
       for (int k = 0; k < 4; ++k) wt[k] = __shfl_sync(0xffffffffu, wown, (lane & ~3) | k);
     } else {
@@ -399,8 +419,8 @@ __device__ __forceinline__ void quantize_tile(const TileOut& o, QuantScratch& sm
       rs_step<8>(s, 16, lane);
       rs_step<4>(s, 8, lane);
       rs_step<2>(s, 4, lane);
-      lt_own = log2_scale(s[0]);
-      const float wown = ex2_fast(-2.f * lt_own);
+      lt_sum = s[0];
+      const float wown = weight_of_sum(s[0]);
 #pragma unroll
       for (int k = 0; k < 8; ++k) wt[k] = __shfl_sync(0xffffffffu, wown, c | (k << 2));
     }
@@ -409,6 +429,7 @@ __device__ __forceinline__ void quantize_tile(const TileOut& o, QuantScratch& sm
   // ---- stored fp16 log-scales and their fp32 multipliers
   const int t_own = (SIDE == 0) ? 16 * (2 * warp + ((lane >> 1) & 1)) + g + 8 * (lane & 1)
                                 : 8 * (4 * warp + (lane >> 3)) + 2 * c + ((lane >> 2) & 1);
+  const float lt_own = log2_scale(lt_sum), lc_own = log2_scale(lc_sum);
   const __half Lt16 = __float2half_rn(lt_own);
   const __half Lc16 = __float2half_rn(lc_own);
   sm.mt[t_own] = __double2float_rn(exp2(-static_cast<double>(__half2float(Lt16))));
