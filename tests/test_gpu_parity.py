@@ -484,3 +484,34 @@ def test_decode_many_short_sequences(K):
     for b, i, j in trip:
         e = np.abs(mq[b, i, j].astype(np.float64) - ref3[b, i, j].astype(np.float64))
         assert np.all(e <= decode_bound(ref3[b, i, j])), (b, i, j)
+
+
+def test_decode_append_consecutive_steps(K):
+    """Five consecutive append steps per sequence (125 -> 130 tokens and
+    252 -> 257, the tiles filling on the way), each against the oracle's step
+    on the GPU's own state before it."""
+    w = inputs.make_decode_workload("steps", [125, 128 + 124], 8, 2, seed=950, pool_blocks=6, max_blocks_per_seq=3)
+    bt = w.block_table.copy()
+    free = [i for i in range(w.num_blocks) if i != int(bt[1, 0])]   # blocks no full tile uses
+    bt[0, 0], bt[0, 1], bt[1, 1], bt[1, 2] = free[:4]               # for the tiles that fill
+    cfg = K.config()
+    packed, scales = K.alloc_cache(cfg, w.num_blocks, 2)
+    if w.k_full.shape[0]:
+        K.quantize_tiles(_dev(w.k_full), _dev(w.v_full), _dev(w.slot_mapping), packed, scales, cfg)
+    tail = _dev(w.tail)
+    lens = w.seq_lens.copy()
+    rng = np.random.default_rng(951)
+    outl = inputs.pick_outlier_channels(np.random.default_rng(952), 2)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for step in range(5):
+        k_new, v_new = inputs.gen_k(rng, 2, 2, outl), inputs.gen_v(rng, 2, 2)
+        p0, s0, t0 = packed.cpu().numpy(), scales.cpu().numpy(), tail.cpu().numpy()
+        out = K.decode_attention_append(_dev(w.q), _dev(k_new), _dev(v_new), packed, scales, tail, _dev(bt),
+                                        _dev(lens), cfg, dev_status=status).cpu().numpy()
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0
+        ref, p2, s2, t2 = O.decode_append(w.q, k_new, v_new, p0, s0, t0, bt, lens, 2, 4, 2)
+        err, bnd, _ = decode_errors(out, ref, [(b, j) for b in range(2) for j in range(8)])
+        assert np.all(err <= bnd), step
+        assert np.array_equal(tail.cpu().numpy(), t2)
+        lens = lens + 1

@@ -467,3 +467,29 @@ def test_multiquery_query_i_is_decode_of_the_prefix_it_sees():
         for b in range(3):
             assert np.array_equal(out[b, i], ref[b])
     assert np.all(out[3] == 0)
+
+
+def test_append_steps_across_a_tile_fill():
+    """Five consecutive steps from 125 to 130 tokens: the tile fills at the
+    third step.  While every token is fp16 the output is textbook attention;
+    after the fill the step reads the packed tile like decode does."""
+    w, _, _, bt, packed, scales = _append_case([125], 4, 2, seed=71, extra_blocks=2)
+    rng = np.random.default_rng(72)
+    outl = inputs.pick_outlier_channels(np.random.default_rng(73), 2)
+    tail, lens = w.tail.copy(), w.seq_lens.copy()
+    rows_k = [w.tail[0, 0, :, :125].transpose(1, 0, 2)]
+    rows_v = [w.tail[0, 1, :, :125].transpose(1, 0, 2)]
+    for step in range(5):
+        k_new = inputs.gen_k(rng, 1, 2, outl)
+        v_new = inputs.gen_v(rng, 1, 2)
+        out, packed, scales, tail = O.decode_append(w.q, k_new, v_new, packed, scales, tail, bt, lens, 2, 4, 2)
+        rows_k.append(k_new)
+        rows_v.append(v_new)
+        L1 = int(lens[0]) + 1
+        if L1 <= 128:      # nothing quantised yet: plain fp16 attention
+            ref = O.decode_uncompressed(w.q, [np.concatenate(rows_k)], [np.concatenate(rows_v)], np.array([L1]), 2)
+        else:              # the first tile is packed now; decode reads the same cache
+            ref = O.decode(w.q, packed, scales, tail, bt, np.array([L1], dtype=np.int32), 2, 4, 2)
+        assert np.array_equal(out, ref), step
+        lens = lens + 1
+    assert int(lens[0]) == 130
