@@ -24,7 +24,7 @@ Sinkhorn-like [hypho, step 3; lehuy, stage 3], (4) asymmetric low-bit
 round-to-nearest with the scales restored when read, keys 4 bit and values
 2 bit by default, "kvarn_k4v2_g128" [hypho, step 4; lehuy, stage 4].
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent (the kernels follow the same ones):
   * H is the unnormalised Sylvester Hadamard matrix, H[i][j] = (-1)^popcount(i&j),
     applied on the right of each token row: R = X H.  H H^T = 128 I, so the
     inverse is H / 128.
@@ -167,7 +167,7 @@ def dequantize(codes, Lt16, Lc16, zero, step) -> np.ndarray:
 
 
 # ---------------------------------------------------------------------------
-# packed layout (this project's definition)
+# packed layout (this project's own definition, written out in code_position)
 # ---------------------------------------------------------------------------
 
 def code_position(side: str, bits: int, t, d):
