@@ -267,6 +267,14 @@ __device__ __forceinline__ void rotate_v(uint32_t xs, int warp, int lane, float 
 
 // ---------------------------------------------------------------- the tile
 
+// K tiles use the V tiles' register layout (rows = channels) through the
+// normalisation -- its reductions move about a quarter fewer words between
+// lanes -- and are transposed to the K fragment order when packed.  0 keeps
+// the K-specific layout (rows = tokens) throughout.
+#ifndef KVARN_Q_K_VLAYOUT
+#define KVARN_Q_K_VLAYOUT 1
+#endif
+
 // Where one tile's results go.
 struct TileOut {
   uint8_t* codes;        // this side's code block (2048 * BITS bytes, 16-byte aligned)
@@ -281,12 +289,13 @@ struct TileOut {
 // rotation is run a second time from the staged tile (same arithmetic).
 template <int SIDE, int BITS, bool STASH>
 __device__ __forceinline__ void quantize_tile(const TileOut& o, QuantScratch& sm, uint32_t xs, uint32_t tmem) {
+  constexpr bool KL = SIDE == 0 && KVARN_Q_K_VLAYOUT == 0;   // the K-specific layout
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, c = lane & 3;
 
   // ---- 2. rotate
   float A[128];
-  if (SIDE == 0) rotate_k(xs, warp, lane, A); else rotate_v(xs, warp, lane, A);
+  if (KL) rotate_k(xs, warp, lane, A); else rotate_v(xs, warp, lane, A);
   // stash R in this warp's 32 TMEM lanes (lane field: bits 31..16, column: 15..0)
   const uint32_t tr = tmem + (static_cast<uint32_t>(32 * warp) << 16);
   if (STASH) {
@@ -302,7 +311,7 @@ __device__ __forceinline__ void quantize_tile(const TileOut& o, QuantScratch& sm
   }
 
   // ---- 3. normalise
-  constexpr int NT = SIDE == 0 ? 4 : 8;   // tokens per thread
+  constexpr int NT = KL ? 4 : 8;   // tokens per thread
   float wt[NT];                           // token weights 2^(-2 lt)
 #pragma unroll
   for (int i = 0; i < NT; ++i) wt[i] = 1.f;
@@ -310,7 +319,7 @@ __device__ __forceinline__ void quantize_tile(const TileOut& o, QuantScratch& sm
 
   for (int it = 0; it < o.iters; ++it) {
     // channel pass: partial sums over this thread's tokens
-    if (SIDE == 0) {
+    if (KL) {
       float s[32];   // index a*4 + nb*2 + rj
 #pragma unroll
       for (int a = 0; a < 8; ++a)
@@ -364,7 +373,7 @@ __device__ __forceinline__ void quantize_tile(const TileOut& o, QuantScratch& sm
     __syncthreads();
 
     // token pass
-    if (SIDE == 0) {
+    if (KL) {
       float2 uu[16];   // (a, nb) -> channels 16a + 8nb + 2c + {0,1}
 #pragma unroll
       for (int a = 0; a < 8; ++a)
@@ -427,7 +436,7 @@ __device__ __forceinline__ void quantize_tile(const TileOut& o, QuantScratch& sm
   }
 
   // ---- stored fp16 log-scales and their fp32 multipliers
-  const int t_own = (SIDE == 0) ? 16 * (2 * warp + ((lane >> 1) & 1)) + g + 8 * (lane & 1)
+  const int t_own = KL ? 16 * (2 * warp + ((lane >> 1) & 1)) + g + 8 * (lane & 1)
                                 : 8 * (4 * warp + (lane >> 3)) + 2 * c + ((lane >> 2) & 1);
   const float lt_own = log2_scale(lt_sum), lc_own = log2_scale(lc_sum);
   const __half Lt16 = __float2half_rn(lt_own);
@@ -449,10 +458,10 @@ __device__ __forceinline__ void quantize_tile(const TileOut& o, QuantScratch& sm
     for (int q = 0; q < 4; ++q) tmem_ld32(tr + 32 * q, Z + 32 * q);
     tmem_wait_ld();
   } else {
-    if (SIDE == 0) rotate_k(xs, warp, lane, Z); else rotate_v(xs, warp, lane, Z);
+    if (KL) rotate_k(xs, warp, lane, Z); else rotate_v(xs, warp, lane, Z);
   }
   float zlo = 3.402823466e38f, zhi = -3.402823466e38f;
-  if (SIDE == 0) {
+  if (KL) {
     float mtv[4];
 #pragma unroll
     for (int ml = 0; ml < 2; ++ml)
@@ -523,19 +532,30 @@ __device__ __forceinline__ void quantize_tile(const TileOut& o, QuantScratch& sm
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       int idx;                             // index of the (h = 0) element; h = 1 is idx + 1
-      if (SIDE == 0) {   // bl = ml*8 + a;  j = ri + 2*nb;  h = rj
+      if (KL) {   // bl = ml*8 + a;  j = ri + 2*nb;  h = rj
         const int ml = bl >> 3, a = bl & 7, nb = j >> 1, ri = j & 1;
         idx = ((ml * 8 + a) * 2 + nb) * 4 + 2 * ri;
-      } else {           // bl = (ntl>>1)*8 + a;  j = ri + 2*(ntl&1);  h = rj
+      } else {    // V layout: bl = (ntl>>1)*8 + a;  j = ri + 2*(ntl&1);  h = rj
         const int ntl = 2 * (bl >> 3) + (j >> 1), a = bl & 7, ri = j & 1;
         idx = (ntl * 8 + a) * 4 + 2 * ri;
       }
       const float2 y = __fmul2_rn(__fadd2_rn(f2(Z[idx], Z[idx + 1]), f2(-zero, -zero)), f2(inv, inv));
       const float2 r = __fadd2_rn(y, f2(kMagic, kMagic));
       // 0 <= y <= 2^b - 1 up to rounding, so rne(y) sits in the low BITS bits of r
-      const int rho = 4 * bl + j;
-      words[rho / PER] = bfi(__float_as_uint(r.x), words[rho / PER], BITS * (rho % PER), BITS);
-      words[rho / PER] = bfi(__float_as_uint(r.y), words[rho / PER], BITS * (rho % PER) + 16, BITS);
+      if (SIDE == 0 && !KL) {
+        // K codes held in the V layout: this lane has (channel g, tokens 2c, 2c+1)
+        // of an 8x8 block; the K fragment wants (token g, channels 2c, 2c+1).
+        // One transpose of the block's 16-bit code pairs, then the K register
+        // j' = (token half) + 2 (channel half) = (j >> 1) + 2 (j & 1).
+        const uint32_t pr = __byte_perm(__float_as_uint(r.x), __float_as_uint(r.y), 0x5410);
+        const uint32_t tr = movmatrix_t(pr);
+        const int rk = 4 * bl + (j >> 1) + 2 * (j & 1);
+        words[rk / PER] |= (tr & static_cast<uint32_t>(LB | (LB << 16))) << (BITS * (rk % PER));
+      } else {
+        const int rho = 4 * bl + j;
+        words[rho / PER] = bfi(__float_as_uint(r.x), words[rho / PER], BITS * (rho % PER), BITS);
+        words[rho / PER] = bfi(__float_as_uint(r.y), words[rho / PER], BITS * (rho % PER) + 16, BITS);
+      }
     }
 
   // ---- 5. store codes (16-byte chunks, lane-interleaved) and the scale record
