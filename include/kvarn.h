@@ -237,7 +237,7 @@ KVARN_API kvarn_status kvarn_decode_attention_multiquery(const void* q, int32_t 
  * library.)  It is meant for callers that cannot allocate device memory
  * themselves -- for instance code running inside another framework's step
  * that owns all allocations, or a host thread that must not call cudaMalloc
- * because that can synchronise the device.  The split-K scratch is instead a
+ * because that can synchronise the device.  The partial-record scratch is instead a
  * file-scope __device__ array of KVARN_NOALLOC_SCRATCH_BYTES (8 MiB) that
  * every GPU loading this library keeps until the process exits.
  *  - Same arguments and results as kvarn_decode_attention, minus workspace.
