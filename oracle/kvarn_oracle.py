@@ -33,9 +33,9 @@ Readings where the pages are silent (the kernels follow the same ones):
     channels first, then tokens.  Mean squares are floored at 2^-48.
   * log-scales are base 2 and stored as fp16 (round to nearest even).
   * one asymmetric (zero, step) pair per tile and per K / V, from the min and
-    max of the normalised tile, stored as fp32.  Codes are round-half-even of
-    (Z - zero) * (1 / step), clamped to [0, 2^b - 1]; that decision is taken
-    in fp32 from the stored fp16 log-scales, as the kernel takes it.
+    max of the normalised tile, stored as fp32.  Z is formed in fp64 from the
+    stored fp16 log-scales, and codes are round-half-even of (Z - zero) / step
+    in fp64 from the stored fp32 zero and step, clamped to [0, 2^b - 1].
   * decode: softmax scale 1/sqrt(128), q head j reads KV head j // (Hq / Hkv);
     the partial last tile of each sequence (seq_len % 128 tokens) is attended
     in fp16 from a separate tail buffer; the output is fp16 (round to nearest).
@@ -43,6 +43,8 @@ The packed byte layout is this project's own (the pages give none); it is
 written out in `code_position` from its definition and nothing else.
 """
 from __future__ import annotations
+
+import functools
 
 import numpy as np
 
@@ -113,32 +115,29 @@ def normalize_logscales(R: np.ndarray, iters: int) -> tuple[np.ndarray, np.ndarr
 # step 4: asymmetric round-to-nearest  [hypho, step 4; lehuy, stage 4]
 # ---------------------------------------------------------------------------
 
-def multipliers(L16: np.ndarray) -> np.ndarray:
-    """fp32 rounding of 2^-L for stored fp16 log-scales L."""
-    return np.exp2(-L16.astype(np.float64)).astype(np.float32)
-
-
-def quantize_given_scales(R32: np.ndarray, Lt16: np.ndarray, Lc16: np.ndarray, bits: int,
+def quantize_given_scales(R: np.ndarray, Lt16: np.ndarray, Lc16: np.ndarray, bits: int,
                           zero: np.float32 | None = None, step: np.float32 | None = None):
-    """Codes of a rotated tile given its stored fp16 log-scales, in fp32.
+    """Codes of a rotated tile given its stored fp16 log-scales, in fp64.
 
-    Z = (R * 2^-Lt) * 2^-Lc; zero = min Z; step = (max Z - zero) / (2^b - 1)
-    (1 if that is 0); code = clamp(rne((Z - zero) * (1 / step)), 0, 2^b - 1).
+    Z = R * 2^-(Lt + Lc) with the stored fp16 log-scales; zero = fp32(min Z);
+    step = fp32((max Z - zero) / (2^b - 1)), taken from that stored zero (1 if
+    it is 0); code = clamp(rne((Z - zero) / step), 0, 2^b - 1), the division
+    and the rounding in fp64 from the stored fp32 zero and step.
     zero / step may be given (to re-derive codes from stored values).
-    Returns (codes int32 [128][128], zero f32, step f32, y f32 [128][128]).
+    Returns (codes int32 [128][128], zero f32, step f32, y f64 [128][128])
+    where y = (Z - zero) / step before rounding.
     """
-    Lb = np.float32(2 ** bits - 1)
-    R32 = R32.astype(np.float32)
-    Z = (R32 * multipliers(Lt16)[:, None]) * multipliers(Lc16)[None, :]
+    Lb = 2 ** bits - 1
+    R = np.asarray(R, dtype=np.float64)
+    Z = R * np.exp2(-(Lt16.astype(np.float64)[:, None] + Lc16.astype(np.float64)[None, :]))
     if zero is None:
-        zero = Z.min()
-        step = np.float32(np.float32(Z.max() - zero) / Lb)
+        zero = np.float32(Z.min())
+        step = np.float32((Z.max() - np.float64(zero)) / Lb)
         if step == 0:
             step = np.float32(1.0)
     zero = np.float32(zero)
     step = np.float32(step)
-    inv = np.float32(np.float32(1.0) / step)
-    y = (Z - zero) * inv
+    y = (Z - np.float64(zero)) / np.float64(step)
     codes = np.clip(np.rint(y), 0, Lb).astype(np.int32)
     return codes, zero, step, y
 
@@ -150,7 +149,7 @@ def quantize_tile(x16: np.ndarray, bits: int, iters: int = 8) -> dict:
     lt, lc = normalize_logscales(R, iters)
     Lt16 = lt.astype(np.float16)
     Lc16 = lc.astype(np.float16)
-    codes, zero, step, y = quantize_given_scales(R.astype(np.float32), Lt16, Lc16, bits)
+    codes, zero, step, y = quantize_given_scales(R, Lt16, Lc16, bits)
     return dict(R=R, lt=lt, lc=lc, Lt=Lt16, Lc=Lc16, codes=codes, zero=zero, step=step, y=y)
 
 
@@ -207,9 +206,18 @@ def side_bytes(bits: int) -> int:
     return TILE * HEAD_DIM * bits // 8
 
 
-def pack_codes(codes: np.ndarray, side: str, bits: int) -> np.ndarray:
+@functools.lru_cache(maxsize=None)
+def _tile_positions(side: str, bits: int):
+    """code_position of every (t, d) of one tile, computed once per layout."""
     t, d = np.meshgrid(np.arange(TILE), np.arange(HEAD_DIM), indexing="ij")
     byte, bit0 = code_position(side, bits, t, d)
+    byte.setflags(write=False)
+    bit0.setflags(write=False)
+    return byte, bit0
+
+
+def pack_codes(codes: np.ndarray, side: str, bits: int) -> np.ndarray:
+    byte, bit0 = _tile_positions(side, bits)
     out = np.zeros(side_bytes(bits), dtype=np.uint8)
     c = codes.astype(np.int64)
     for b in range(bits):
@@ -219,8 +227,7 @@ def pack_codes(codes: np.ndarray, side: str, bits: int) -> np.ndarray:
 
 
 def unpack_codes(buf: np.ndarray, side: str, bits: int) -> np.ndarray:
-    t, d = np.meshgrid(np.arange(TILE), np.arange(HEAD_DIM), indexing="ij")
-    byte, bit0 = code_position(side, bits, t, d)
+    byte, bit0 = _tile_positions(side, bits)
     return ((buf[byte].astype(np.int64) >> bit0) & ((1 << bits) - 1)).astype(np.int32)
 
 
@@ -404,9 +411,10 @@ def decode_multiquery(q, packed, scales, tail, block_table, seq_lens, num_kv_hea
     Reading (the pages quote time-to-first-token but fix no multi-query
     kernel): q is [B][qlen][Hq][128] fp16; query i of sequence b sits at
     position L - qlen + i (L = seq_lens[b], counting the queries' own tokens)
-    and attends keys [0, L - qlen + i], read as decode reads them.  Defined
-    when L >= qlen and (L % 128) + 1 >= qlen (every query at or after the last
-    full tile's final token); other sequences, and empty ones, give 0.
+    and attends keys [0, L - qlen + i], each read as decode reads it: keys of
+    full tiles dequantised from the packed cache (also when the query sits
+    inside that tile), the last L % 128 from the fp16 tail.  Defined when
+    L >= qlen; other sequences, and empty ones, give 0.
     `heads`: optional (b, i, j) triples to compute.  Returns [B][qlen][Hq][128] fp16.
     """
     B, qlen, Hq, _ = q.shape
@@ -418,7 +426,7 @@ def decode_multiquery(q, packed, scales, tail, block_table, seq_lens, num_kv_hea
     cache = {}
     for b, i, j in trip:
         L = int(seq_lens[b])
-        if L < qlen or (L % TILE) + 1 < qlen or L == 0:
+        if L < qlen or L == 0:
             continue
         K, V = gather_kv(packed, scales, tail, block_table, L, b, j // G, kb, vb, cache)
         lim = L - qlen + i + 1
