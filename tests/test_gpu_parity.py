@@ -6,11 +6,14 @@ Quantizer, staged as in the tolerance plan:
   2. stored fp16 log-scales: the fp16 rounding of some value within that
      tolerance of the oracle's fp64 value (at a rounding boundary either
      neighbour is correct);
-  3. codes re-derived by the oracle (fp32, its own exact rotation) from the
-     GPU's stored scales, zero and step: every mismatch is +-1 at a rounding
-     tie, within the fp32 error bound of the GPU's rotation;
+  3. codes re-derived by the oracle (fp64 decision, its own exact rotation)
+     from the GPU's stored scales, zero and step: >= 99.99 % identical, and
+     every mismatch is +-1 at a rounding tie, within the error bound of the
+     GPU's fp32 arithmetic;
   4. end-to-end codes >= 99.99 % identical to the oracle's own where the
-     stored scales and grid agree (all codes, for <= 4-bit codes).
+     stored row and column scales agree (all widths), and over all codes for
+     <= 4-bit codes; a stored scale may differ only where the oracle's value
+     lies within the stage-1 tolerance of an fp16 rounding boundary.
 Decode: <= 2e-3 absolute (one fp16 step where |o| >= 4 makes that step
 larger) against the oracle's explicit-dequant attention over the GPU's own
 packed cache (read through the oracle's own unpacker).
@@ -71,6 +74,18 @@ def _fp16_neighbours_ok(gpu16, x64, tol=LOG_TOL):
     return (g >= lo) & (g <= hi)
 
 
+def stage3_bound(x, Lt, Lc, zero, step, y):
+    """How far the kernel's fp32 value of (Z - zero) / step may lie from the
+    oracle's fp64 one: the kernel's fp32 rotation (error below 2^-18 of the
+    row's absolute sum), Z formed with two fp32 products of fp32 multipliers,
+    the subtraction of zero and the product with the fp32 reciprocal of step."""
+    mt = np.exp2(-Lt.astype(np.float64))[:, None]
+    mc = np.exp2(-Lc.astype(np.float64))[None, :]
+    dR = 2.0 ** -18 * np.abs(x.astype(np.float64)).sum(axis=1)[:, None]
+    Z = np.float64(zero) + np.float64(step) * y
+    return (dR * mt * mc + 2.0 ** -21 * (np.abs(Z) + abs(float(zero)))) / float(step) + 2.0 ** -21 * np.abs(y)
+
+
 def check_tile(x, bits, codes, Lt, Lc, zero, step, cnt, lt_gpu=None, lc_gpu=None, where=()):
     """Stages 1-4 for one tile x ([128][128] fp16) against the GPU's stored
     codes / Lt / Lc / zero / step (stage 1 only with the GPU's fp32
@@ -84,36 +99,43 @@ def check_tile(x, bits, codes, Lt, Lc, zero, step, cnt, lt_gpu=None, lc_gpu=None
     # stage 2
     assert np.all(_fp16_neighbours_ok(Lt, r["lt"])), where
     assert np.all(_fp16_neighbours_ok(Lc, r["lc"])), where
-    # stage 3: codes given the GPU's stored scales, zero and step
-    R32 = r["R"].astype(np.float32)
-    c_given, z2, s2, y = O.quantize_given_scales(R32, Lt, Lc, bits)
-    assert abs(float(z2) - float(zero)) <= 1e-6 * max(1.0, abs(float(zero))) + 1e-30, (z2, zero)
-    assert abs(float(s2) - float(step)) <= 1e-6 * float(s2), (s2, step)
-    c_g, _, _, y_g = O.quantize_given_scales(R32, Lt, Lc, bits, zero, step)
+    # stage 3: the oracle's fp64 code decision given the GPU's stored scales;
+    # its own zero / step from those scales agree with the GPU's to fp32 rounding
+    c_given, z2, s2, _ = O.quantize_given_scales(r["R"], Lt, Lc, bits)
+    assert abs(float(z2) - float(zero)) <= 2e-6 * max(1.0, abs(float(zero))), (z2, zero)
+    assert abs(float(s2) - float(step)) <= 2e-6 * float(s2), (s2, step)
+    c_g, _, _, y_g = O.quantize_given_scales(r["R"], Lt, Lc, bits, zero, step)
     diff = codes != c_g
     if diff.any():
         assert np.all(np.abs(codes[diff] - c_g[diff]) == 1)
-        mt = O.multipliers(Lt).astype(np.float64)[:, None]
-        mc = O.multipliers(Lc).astype(np.float64)[None, :]
-        dR = 2.0 ** -18 * np.abs(x.astype(np.float64)).sum(axis=1)[:, None]
-        dy = dR * mt * mc / float(step) + 2.0 ** -20 * np.abs(y_g)
+        dy = stage3_bound(x, Lt, Lc, zero, step, y_g)
         frac = np.abs(y_g - np.floor(y_g) - 0.5)
         assert np.all(frac[diff] <= dy[diff]), (where, frac[diff].max())
-    # stage 4: end to end.  Where a stored scale (or the tile's grid)
-    # legitimately differs from the oracle's at a rounding boundary, stage 3
-    # has already validated the codes; the unique part is the elements whose
-    # scales and grid agree.
+    # stage 4: end to end against the oracle's own codes.  A stored log-scale
+    # the GPU rounded to the other fp16 neighbour (stage 2 allows it at a
+    # rounding boundary) moves the codes of its whole row or column, and both
+    # results are correct; the unique part is the codes whose row and column
+    # scales agree.
     e2e = codes != r["codes"]
-    same = (Lt == r["Lt"])[:, None] & (Lc == r["Lc"])[None, :]
-    if not (zero == r["zero"] and step == r["step"]):
-        same[:] = False
+    flips_t = Lt != r["Lt"]
+    flips_c = Lc != r["Lc"]
+    same = (~flips_t)[:, None] & (~flips_c)[None, :]
+    window_t = (r["lt"] - LOG_TOL).astype(np.float16) != (r["lt"] + LOG_TOL).astype(np.float16)
+    window_c = (r["lc"] - LOG_TOL).astype(np.float16) != (r["lc"] + LOG_TOL).astype(np.float16)
     for k, v in (("mism_given", int(diff.sum())), ("mism_e2e", int(e2e.sum())), ("total", codes.size),
-                 ("mism_same", int((e2e & same).sum())), ("total_same", int(same.sum()))):
+                 ("mism_same", int((e2e & same).sum())), ("total_same", int(same.sum())),
+                 ("scale_flips", int(flips_t.sum() + flips_c.sum())), ("scales", 256),
+                 ("scale_window", int(window_t.sum() + window_c.sum()))):
         cnt[k] = cnt.get(k, 0) + v
 
 
 def assert_counts(cnt, kb, vb):
+    """>= 99.99 % of codes bit-exact where the scales agree (all widths) and
+    over all codes for <= 4-bit codes; the re-derived codes of stage 3 too;
+    stored scales flip only inside the rounding-boundary window."""
+    assert cnt["mism_given"] <= 1e-4 * cnt["total"], cnt
     assert cnt["mism_same"] <= 1e-4 * cnt["total_same"], cnt
+    assert cnt["scale_flips"] <= cnt["scale_window"], cnt
     if max(kb, vb) <= 4:
         assert cnt["mism_e2e"] <= 1e-4 * cnt["total"], cnt
 
@@ -135,8 +157,7 @@ def check_quantize_parity(K, k, v, slot, num_blocks, kb, vb, groups=None, report
                            dbg[g, h, sidx, :128].astype(np.float64), dbg[g, h, sidx, 128:].astype(np.float64),
                            where=(g, h, side))
     if report is not None:
-        report.update(total=cnt["total"], mism_e2e=cnt["mism_e2e"], mism_given=cnt["mism_given"],
-                      worst_scale=cnt["worst_scale"], total_same=cnt["total_same"], mism_same=cnt["mism_same"])
+        report.update(cnt)
     assert_counts(cnt, kb, vb)
     return packed, scales
 
@@ -383,29 +404,108 @@ def test_decode_append_status(K):
 
 def test_full_size_qwen3_32b_sampled(K):
     """The Qwen3-32B-shaped workload (B=8, 16K + ragged tail, 64/8 heads) in the
-    bench's launch configuration: all tiles quantised and decoded on the GPU,
-    a sample of tiles and outputs checked against the oracle."""
+    bench's launch configuration: every tile quantised and decoded on the
+    GPU.  The quantiser is checked through stages 1-4 on 256 sampled tiles
+    (16 token groups x all 8 KV heads x K and V) with the contract's bounds;
+    the decode on sampled outputs, including every head of one sequence."""
     w = inputs.qwen3_32b()
     cfg = K.config()
     packed, scales = K.alloc_cache(cfg, w.num_blocks, w.num_kv_heads)
     dbg = torch.zeros((w.k_full.shape[0] // 128, 8, 2, 256), dtype=torch.float32, device="cuda")
-    K.quantize_tiles(_dev(w.k_full), _dev(w.v_full), _dev(w.slot_mapping), packed, scales, cfg, debug_logscales=dbg)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    K.quantize_tiles(_dev(w.k_full), _dev(w.v_full), _dev(w.slot_mapping), packed, scales, cfg, dev_status=status,
+                     debug_logscales=dbg)
     out, packed_h, scales_h = run_decode(K, w, packed=packed, scales=scales)
+    assert int(status.item()) == 0
+    dbg_h = dbg.cpu().numpy()
     rng = np.random.default_rng(5)
     n_groups = w.k_full.shape[0] // 128
-    for g in rng.choice(n_groups, size=6, replace=False):
+    cnt = {}
+    for g in rng.choice(n_groups, size=16, replace=False):
         blk = int(w.slot_mapping[g * 128]) // 128
-        for h in (0, 5):
-            for side, src, bits in (("K", w.k_full, 4), ("V", w.v_full, 2)):
-                r = O.quantize_tile(np.ascontiguousarray(src[g * 128:(g + 1) * 128, h]), bits, 8)
+        for h in range(8):
+            for sidx, side, src, bits in ((0, "K", w.k_full, 4), (1, "V", w.v_full, 2)):
+                x = np.ascontiguousarray(src[g * 128:(g + 1) * 128, h])
                 codes, Lt, Lc, z, s = O.read_tile(packed_h, scales_h, blk, h, side, 4, 2)
-                assert (codes != r["codes"]).mean() <= 1e-3
-                assert np.all(_fp16_neighbours_ok(Lt, r["lt"]))
-    heads = [(0, 0), (3, 17), (7, 63)]
+                check_tile(x, bits, codes, Lt, Lc, z, s, cnt, dbg_h[g, h, sidx, :128].astype(np.float64),
+                           dbg_h[g, h, sidx, 128:].astype(np.float64), where=(int(g), h, side))
+    print(f"full size k4v2, 256 tiles: {cnt}")
+    assert cnt["total"] == 256 * 128 * 128
+    assert_counts(cnt, 4, 2)
+    heads = [(0, 0), (3, 17), (7, 63), (5, 40)] + [(2, j) for j in range(64)]
     ref = O.decode(w.q, packed_h, scales_h, w.tail, w.block_table, w.seq_lens, 8, 4, 2, heads=heads)
     err, bnd, _ = decode_errors(out, ref, heads)
+    print(f"full size decode: max err {err.max():.2e} over {len(heads)} outputs")
     assert np.all(err <= bnd)
     assert np.all(np.isfinite(out.astype(np.float32)))
+
+
+def test_llama3_8b_config_decode_all_outputs(K):
+    """The Llama-3-8B-shaped decode (B=16, 4096 tokens each, 32/8 heads,
+    shuffled 512-block pool): every output against the oracle over the GPU's
+    own cache."""
+    w = inputs.llama3_8b()
+    err, _ = check_decode(K, w)
+    print(f"llama3_8b B16 x 4K: max abs err {err:.2e}")
+
+
+def test_llama3_70b_config_decode_sampled(K):
+    """The Llama-3-70B-shaped long-context decode (B=4, lengths U[1024,
+    131072] from the seed, 64/8 heads): 16 sampled outputs, 4 per sequence
+    over 2 KV heads each, the longest sequence included, against the oracle
+    over the GPU's own cache."""
+    w = inputs.llama3_70b()
+    assert int(w.seq_lens.max()) > 100_000
+    out, packed_h, scales_h = run_decode(K, w)
+    rng = np.random.default_rng(6)
+    worst = 0.0
+    for b in range(w.num_seqs):
+        for h in rng.choice(8, size=2, replace=False):
+            heads = [(b, int(h) * 8 + int(j)) for j in rng.choice(8, size=2, replace=False)]
+            ref = O.decode(w.q, packed_h, scales_h, w.tail, w.block_table, w.seq_lens, 8, 4, 2, heads=heads)
+            err, bnd, _ = decode_errors(out, ref, heads)
+            assert np.all(err <= bnd), (b, int(h))
+            worst = max(worst, float(err.max()))
+    print(f"llama3_70b lengths {w.seq_lens.tolist()}: max abs err {worst:.2e}")
+
+
+def test_tensor_parallel_kv_head_shards_on_gpu(K):
+    """Tensor parallelism over KV heads (the pages' TP=2 setting, [hypho]
+    这就是 KVarN 想解决的问题): each of two shards quantises and decodes only
+    its own KV heads and the query heads that read them, on its own cache
+    slice, through the CUDA path; the concatenated outputs equal the oracle's
+    decode of the whole problem."""
+    from bit_kv_cache_15_b200.sharding import kv_head_shard
+    w = inputs.make_decode_workload("tp", [9 * 128 + 70, 3 * 128, 200, 20 * 128 + 1], 32, 8, seed=960,
+                                    pool_blocks=40)
+    cfg = K.config()
+    out = np.zeros_like(w.q)
+    caches = []
+    for rank in range(2):
+        kv, qh = kv_head_shard(8, 32, rank, 2)
+        ks, qs = slice(kv.start, kv.stop), slice(qh.start, qh.stop)
+        packed, scales = K.alloc_cache(cfg, w.num_blocks, len(kv))
+        status = torch.zeros(1, dtype=torch.int32, device="cuda")
+        K.quantize_tiles(_dev(w.k_full[:, ks]), _dev(w.v_full[:, ks]), _dev(w.slot_mapping), packed, scales, cfg,
+                         dev_status=status)
+        o = K.decode_attention(_dev(w.q[:, qs]), packed, scales, _dev(w.tail[:, :, ks]), _dev(w.block_table),
+                               _dev(w.seq_lens), cfg, dev_status=status)
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0
+        out[:, qs] = o.cpu().numpy()
+        caches.append((packed.cpu().numpy(), scales.cpu().numpy()))
+    packed_all = np.concatenate([c[0] for c in caches], axis=1)
+    scales_all = np.concatenate([c[1] for c in caches], axis=1)
+    ref = O.decode(w.q, packed_all, scales_all, w.tail, w.block_table, w.seq_lens, 8, 4, 2)
+    err, bnd, _ = decode_errors(out, ref, [(b, j) for b in range(w.num_seqs) for j in range(32)])
+    print(f"TP=2 over KV heads: max abs err {err.max():.2e}")
+    assert np.all(err <= bnd)
+    # each shard's cache is the whole problem's cache for its heads
+    ref_p, ref_s = O.quantize_tiles(w.k_full, w.v_full, w.slot_mapping, 8, w.num_blocks, 4, 2,
+                                    groups=range(2))
+    blk = [int(w.slot_mapping[g * 128]) // 128 for g in range(2)]
+    mism = float((packed_all[blk] != ref_p[blk]).mean())
+    assert mism < 1e-3, mism
 
 
 @pytest.mark.parametrize("lens,hq,hkv,heads", [
@@ -428,13 +528,15 @@ def test_decode_long_ragged_sampled(K, lens, hq, hkv, heads):
 
 # ------------------------------------------------------------------ multi-query
 
-@pytest.mark.parametrize("hq,hkv,qlen", [(64, 8, 4), (8, 8, 3), (16, 2, 2), (8, 2, 1)])
+@pytest.mark.parametrize("hq,hkv,qlen", [(64, 8, 4), (8, 8, 3), (16, 2, 2), (8, 2, 1), (8, 8, 128), (16, 2, 37)])
 def test_decode_multiquery_parity(K, hq, hkv, qlen):
     """q_len queries per sequence, causal: (query, head) columns in groups of
-    8 per KV head (4 groups at 64/8 heads x 4 queries).  Lengths cover a query
-    block ending a full tile, a tail-only sequence, long sequences and one
-    that breaks the precondition (tail shorter than q_len - 1)."""
-    lens = [256 + qlen - 1, 1024 + 127, 40 * 128 + 10, 7 + qlen, 128 + max(qlen - 2, 0), 3 * 128 + 50]
+    8 per KV head (4 groups at 64/8 heads x 4 queries, 128 at 8/8 x 128).
+    Lengths cover a query block ending a full tile, queries inside the last
+    full tile (tail shorter than q_len - 1, or no tail at all), a tail-only
+    sequence, long sequences and one shorter than q_len."""
+    lens = [256 + qlen - 1, 1024 + 127, 40 * 128 + 10, 7 + qlen, 128 + max(qlen - 2, 0), 3 * 128 + 50,
+            5 * 128, 2 * 128 + 1, max(qlen - 1, 0)]
     full = sum(L // 128 for L in lens)
     w = inputs.make_decode_workload("mq", lens, hq, hkv, seed=800 + qlen, pool_blocks=full + 2)
     cfg = K.config()
@@ -445,13 +547,16 @@ def test_decode_multiquery_parity(K, hq, hkv, qlen):
     out = K.decode_attention_multiquery(_dev(q), packed, scales, _dev(w.tail), _dev(w.block_table), _dev(w.seq_lens),
                                         cfg, dev_status=status).cpu().numpy()
     torch.cuda.synchronize()
-    bad = [b for b, L in enumerate(lens) if not (L >= qlen and L % 128 + 1 >= qlen)]
+    bad = [b for b, L in enumerate(lens) if L < qlen]
     assert int(status.item()) == (3 if bad else 0)
+    inside = [b for b, L in enumerate(lens) if L >= qlen and L >= 128 and L % 128 + 1 < qlen]
+    if qlen > 2:
+        assert inside, "some sequence must place queries inside its last full tile"
     ref = O.decode_multiquery(q, packed.cpu().numpy(), scales.cpu().numpy(), w.tail, w.block_table, w.seq_lens,
                               hkv, 4, 2)
     err = np.abs(out.astype(np.float64) - ref.astype(np.float64))
     bnd = decode_bound(ref)
-    print(f"multiquery {hq}/{hkv} q_len={qlen}: max err {err.max():.2e}")
+    print(f"multiquery {hq}/{hkv} q_len={qlen}: max err {err.max():.2e} (inside a packed tile: {inside})")
     assert np.all(err <= bnd)
     for b in bad:
         assert np.all(out[b] == 0)
@@ -471,7 +576,7 @@ def test_decode_many_short_sequences(K):
     err, bnd, _ = decode_errors(out, ref, heads)
     assert np.all(err <= bnd)
     assert np.all(out[7] == 0)
-    # the same cache read as 3-query verify steps (sequences with < 2 tail rows give 0)
+    # the same cache read as 3-query verify steps (sequences shorter than 3 give 0)
     cfg = K.config()
     q = rng.standard_normal((100, 3, 4, 128)).astype(np.float16)
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
