@@ -390,7 +390,8 @@ cudaError_t launch_b(const BaselineArgs& p, cudaStream_t stream) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  const uint64_t bit = 1ull << (dev & 63);
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;   // one configured bit per ordinal
+  const uint64_t bit = 1ull << dev;
   if ((configured.load(std::memory_order_acquire) & bit) == 0) {
     e = cudaFuncSetAttribute(baseline_kernel<FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, T::kSmem);
     if (e != cudaSuccess) return e;

@@ -19,8 +19,12 @@ constexpr int kHeadDim = 128;
 constexpr int kScaleRec = KVARN_SCALE_RECORD_BYTES;  // 528
 constexpr float kLog2e = 1.4426950408889634f;
 
-// Bounded spin on an mbarrier: ~2^26 polls (far above any copy latency).
-constexpr uint32_t kWaitLimit = 1u << 26;
+// Bounded spin on an mbarrier: ~2^26 polls (far above any copy latency).  A
+// test build may lower it to exercise the timeout status.
+#ifndef KVARN_WAIT_LIMIT_LOG2
+#define KVARN_WAIT_LIMIT_LOG2 26
+#endif
+constexpr uint32_t kWaitLimit = 1u << KVARN_WAIT_LIMIT_LOG2;
 
 __device__ __forceinline__ void report_status(int32_t* st, int code) {
   if (st != nullptr) atomicCAS(st, 0, code);

@@ -361,6 +361,14 @@ __device__ __forceinline__ bool issue_unit(const DecodeArgs& p, uint8_t* stage_b
   if (lane == 0) {
     uint8_t* dst = stage_base + (k & 1) * T::kStage;
     uint64_t* bar = &my_bars[k & 1];
+#if KVARN_TEST_STALL_FIRST_UNIT
+    // test build only: the first unit of warp 0 of CTA 0 expects 16 bytes that
+    // are never sent and no copy is issued, so its bounded wait runs out
+    if (blockIdx.x == 0 && threadIdx.x == 0 && k == 0) {
+      mbar_arrive_expect_tx(bar, 16);
+      return ok;
+    }
+#endif
     if (ok) {
       const uint8_t* cb = p.packed + ((int64_t)blk * p.Hkv + h) * T::kCode;
       mbar_arrive_expect_tx(bar, T::kStage);
@@ -376,14 +384,17 @@ __device__ __forceinline__ bool issue_unit(const DecodeArgs& p, uint8_t* stage_b
   return ok;
 }
 
-// One segment: full tiles [t_begin, t_end) of sequence b, KV head h, by the
-// whole CTA; writes one partial record per query head at recs + g * 132.
+// One segment: full tiles [t_begin, t_end) of sequence b (length L), KV head
+// h, by the whole CTA; writes one partial record per query head at
+// recs + g * 132.  With several queries per sequence the last full tile can
+// hold query positions: there each (query, head) column masks the tokens
+// after its own query.
 // Work units (tile, part) go round-robin over the warps starting at warp
 // `woff`, so a CTA that runs several segments keeps its warps level.  `rearm`:
 // the barriers were used by an earlier segment and are invalidated first.
 // Returns false if a copy timed out (the status is set).
 template <int KB, int VB>
-__device__ __forceinline__ bool decode_segment(const DecodeArgs& p, uint8_t* smem, int b, int h, int grp,
+__device__ __forceinline__ bool decode_segment(const DecodeArgs& p, uint8_t* smem, int b, int h, int grp, int L,
                                                int t_begin, int t_end, int woff, bool rearm, float* recs) {
   using T = DecodeTraits<KB, VB>;
   constexpr int U = T::U, MT = T::MT;
@@ -467,6 +478,18 @@ __device__ __forceinline__ bool decode_segment(const DecodeArgs& p, uint8_t* sme
     qr[4 * kt + 3] = hi.y;
   }
 #endif
+  // causal limits (last token index attended inside the last full tile) of
+  // this lane's columns 2c, 2c + 1: query i sits at position L - qlen + i
+  const int mask_tile = p.qlen > 1 ? (L >> 7) - 1 : -1;
+  int climit[2] = {kTile - 1, kTile - 1};
+  if (mask_tile >= 0) {
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      int64_t row;
+      int qi;
+      if (col_row(p, b, h, grp, 2 * c + j, &row, &qi)) climit[j] = L - p.qlen + qi - kTile * mask_tile;
+    }
+  }
   const float coef0 = p.sm_scale * kLog2e * (1.f / 128.f) * invsig[2 * c];
   const float coef1 = p.sm_scale * kLog2e * (1.f / 128.f) * invsig[2 * c + 1];
   float* scr = reinterpret_cast<float*>(smem + T::kScrOff) + warp * kHeadDim;
@@ -622,6 +645,25 @@ __device__ __forceinline__ bool decode_segment(const DecodeArgs& p, uint8_t* sme
         mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
         mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
       }
+      if (t_begin + (u0 + k * kDWarps) / U == mask_tile) {   // warp-uniform: the tile holding query positions
+        mx0 = -INFINITY;
+        mx1 = -INFINITY;
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+          for (int ri = 0; ri < 2; ++ri) {
+            const int t = t0 + 16 * mt + g8 + 8 * ri;
+            if (t > climit[0]) S[mt][2 * ri] = -INFINITY;
+            if (t > climit[1]) S[mt][2 * ri + 1] = -INFINITY;
+            mx0 = fmaxf(mx0, S[mt][2 * ri]);
+            mx1 = fmaxf(mx1, S[mt][2 * ri + 1]);
+          }
+#pragma unroll
+        for (int o = 4; o < 32; o <<= 1) {
+          mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+          mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+        }
+      }
       // V token scales relative to the tile's largest, times 2^kPBoost: the weights
       // p * tv fed to the mma then stay in fp16's normal range down to p * tv ~ 2^-26
       // of the tile maximum; the common factor is undone on the fold below
@@ -637,7 +679,10 @@ __device__ __forceinline__ bool decode_segment(const DecodeArgs& p, uint8_t* sme
 #pragma unroll
         for (int ri = 0; ri < 2; ++ri) tv[mt][ri] = ex2_fast(tv[mt][ri] - lvm + static_cast<float>(kPBoost));
       const float mn0 = fmaxf(mrun[0], mx0), mn1 = fmaxf(mrun[1], mx1);
-      const float al0 = ex2_fast(mrun[0] - mn0), al1 = ex2_fast(mrun[1] - mn1);
+      // a column that has attended no token yet (masked) keeps max -inf: its
+      // exponents are taken against 0, so its weights are 0 instead of NaN
+      const float e0 = mn0 == -INFINITY ? 0.f : mn0, e1 = mn1 == -INFINITY ? 0.f : mn1;
+      const float al0 = ex2_fast(mrun[0] - e0), al1 = ex2_fast(mrun[1] - e1);
       mrun[0] = mn0;
       mrun[1] = mn1;
       float ls0 = 0.f, ls1 = 0.f, ps0 = 0.f, ps1 = 0.f;
@@ -647,8 +692,8 @@ __device__ __forceinline__ bool decode_segment(const DecodeArgs& p, uint8_t* sme
         uint32_t pk[2];
 #pragma unroll
         for (int ri = 0; ri < 2; ++ri) {
-          const float p0 = ex2_fast(S[mt][2 * ri] - mn0);
-          const float p1 = ex2_fast(S[mt][2 * ri + 1] - mn1);
+          const float p0 = ex2_fast(S[mt][2 * ri] - e0);
+          const float p1 = ex2_fast(S[mt][2 * ri + 1] - e1);
           ls0 += p0;
           ls1 += p1;
           const __half2 hp = __floats2half2_rn(p0 * tv[mt][ri], p1 * tv[mt][ri]);
@@ -792,10 +837,10 @@ __device__ __forceinline__ bool decode_segment(const DecodeArgs& p, uint8_t* sme
 constexpr int kTailUnits = 9;
 constexpr int kFillUnits = 16;
 
-// With qlen > 1 the queries must lie at or after the last full tile's final
-// token ((L mod 128) + 1 >= qlen), so that only the fp16 tail needs causal masks.
+// With qlen > 1 the sequence must hold its qlen query tokens (L >= qlen); as
+// qlen <= 128, query positions reach back at most into the last full tile.
 __device__ __forceinline__ bool seq_valid(const DecodeArgs& p, int L) {
-  return L >= 0 && L + p.append <= kTile * p.max_blocks && (p.qlen == 1 || (L >= p.qlen && (L & 127) + 1 >= p.qlen));
+  return L >= 0 && L + p.append <= kTile * p.max_blocks && (p.qlen == 1 || L >= p.qlen);
 }
 __device__ __forceinline__ int pair_tiles(int L, bool valid) { return valid ? (L >> 7) : 0; }
 __device__ __forceinline__ int pair_units(const DecodeArgs& p, int L, bool valid) {
@@ -1055,7 +1100,7 @@ __global__ void __launch_bounds__(kDThreads, KVARN_D_MIN_CTAS) decode_kernel(con
     const int h = sp / p.ngrp, grp = sp - (sp / p.ngrp) * p.ngrp;
     const int pair = b * p.Hkv * p.ngrp + sp;
     if (ok && t_a < t_e) {
-      ok = decode_segment<KB, VB>(p, smem, b, h, grp, t_a, t_e, woff, rearm,
+      ok = decode_segment<KB, VB>(p, smem, b, h, grp, L, t_a, t_e, woff, rearm,
                                   p.ws + static_cast<int64_t>(pair + cta) * p.C * kPartialFloats);
       rearm = true;
       woff = (woff + (t_e - t_a) * DecodeTraits<KB, VB>::U) % kDWarps;
@@ -1091,7 +1136,8 @@ cudaError_t launch_d(const DecodeArgs& p, cudaStream_t stream) {
   int dev = 0;
   cudaError_t e0 = cudaGetDevice(&dev);
   if (e0 != cudaSuccess) return e0;
-  const uint64_t bit = 1ull << (dev & 63);
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;   // one configured bit per ordinal
+  const uint64_t bit = 1ull << dev;
   if ((configured.load(std::memory_order_acquire) & bit) == 0) {
     cudaError_t e = cudaFuncSetAttribute(decode_kernel<KB, VB>, cudaFuncAttributeMaxDynamicSharedMemorySize, T::kSmem);
     if (e != cudaSuccess) return e;
@@ -1099,22 +1145,25 @@ cudaError_t launch_d(const DecodeArgs& p, cudaStream_t stream) {
     e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
     const int n = KVARN_D_MIN_CTAS * sms;
-    ctas[dev & 63] = n < 1 ? 1 : (n > kDecodeMaxCtas ? kDecodeMaxCtas : n);
+    ctas[dev] = n < 1 ? 1 : (n > kDecodeMaxCtas ? kDecodeMaxCtas : n);
     configured.fetch_or(bit, std::memory_order_acq_rel);
   }
   // the per-(seq, KV head) unit counters start every call at zero
   cudaError_t e = cudaMemsetAsync(p.counters, 0, static_cast<size_t>(p.B) * p.Hkv * p.ngrp * sizeof(int), stream);
   if (e != cudaSuccess) return e;
-  decode_kernel<KB, VB><<<ctas[dev & 63], kDThreads, T::kSmem, stream>>>(p);
+  decode_kernel<KB, VB><<<ctas[dev], kDThreads, T::kSmem, stream>>>(p);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 // ------------------------------------------------------------------ fixed scratch
-// Device-resident scratch for kvarn_decode_attention_noalloc: the split-K
-// partial records live in this file-scope array instead of a caller-supplied
-// workspace.  Every GPU that loads the library holds these bytes until exit.
+// Device-resident scratch for kvarn_decode_attention_noalloc: the stream-K
+// partial records and arrival counters live in this file-scope array instead
+// of a caller-supplied workspace.  Every GPU that loads the library holds these
+// bytes until exit.  Its device address is looked up once per device ordinal
+// and cached for the life of the process: after a reset of the device's
+// primary context (cudaDeviceReset) the cached address is stale.
 static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchBytes / sizeof(float)];
 
 cudaError_t noalloc_scratch(void** ptr, size_t* bytes) {

@@ -192,7 +192,8 @@ cudaError_t launch_q(const QuantArgs& p, cudaStream_t stream) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  const uint64_t bit = 1ull << (dev & 63);
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;   // one configured bit per ordinal
+  const uint64_t bit = 1ull << dev;
   const int smem = static_cast<int>(sizeof(QuantSmem));
   if ((configured.load(std::memory_order_acquire) & bit) == 0) {
     e = cudaFuncSetAttribute(quantize_kernel<KB, VB>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -204,8 +205,8 @@ cudaError_t launch_q(const QuantArgs& p, cudaStream_t stream) {
     e = resident_ctas(reinterpret_cast<const void*>(quantize_kernel<KB, VB>), smem, dev, &occ);
     if (e != cudaSuccess) return e;
     // each resident CTA holds kTmemCols of the SM's 512 tensor-memory columns
-    ctas_per_sm[dev & 63] = occ < 1 ? 1 : (occ > kMaxCtasPerSm ? kMaxCtasPerSm : occ);
-    sms[dev & 63] = n;
+    ctas_per_sm[dev] = occ < 1 ? 1 : (occ > kMaxCtasPerSm ? kMaxCtasPerSm : occ);
+    sms[dev] = n;
     configured.fetch_or(bit, std::memory_order_acq_rel);
   }
   CUtensorMap mk, mv;
@@ -214,7 +215,7 @@ cudaError_t launch_q(const QuantArgs& p, cudaStream_t stream) {
   e = make_map(&mv, p.v, p.hkv, p.num_groups * kTile);
   if (e != cudaSuccess) return e;
   const int64_t tiles = 2 * p.num_groups * p.hkv;
-  const int64_t slots = static_cast<int64_t>(sms[dev & 63]) * ctas_per_sm[dev & 63];
+  const int64_t slots = static_cast<int64_t>(sms[dev]) * ctas_per_sm[dev];
   const unsigned grid = static_cast<unsigned>(tiles < slots ? tiles : slots);
   quantize_kernel<KB, VB><<<grid, kQThreads, smem, stream>>>(mk, mv, p);
   return cudaGetLastError();

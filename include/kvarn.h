@@ -20,6 +20,10 @@
  *    allocates no memory and keeps no state between calls.
  *  - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
  *    stream) and the call returns without synchronising.  Calls are reentrant.
+ *  - Each kernel's launch set-up (its shared-memory attribute and grid size)
+ *    is done once per device ordinal (ordinals 0-63; others get
+ *    KVARN_ERR_CUDA) and kept for the process; a reset of the device's primary
+ *    context (cudaDeviceReset) is not supported while the library is in use.
  *  - Argument and shape errors are found on the host and returned before any
  *    launch.  A launch failure returns KVARN_ERR_CUDA.
  *  - Data-dependent faults found on the device (a slot or block id out of
@@ -203,22 +207,23 @@ KVARN_API kvarn_status kvarn_decode_attention_append(const void* q, const void* 
 
 /* Multi-query attention over the packed cache: q_len query tokens per
  * sequence, each attending causally -- the shape of a speculative-decoding
- * verify step or a short chunk of chunked prefill.  The pages quote
- * time-to-first-token figures but give no kernel for it; this is the decode
- * path with (query, head) columns in place of heads.
+ * verify step or a chunk of chunked prefill.  The pages quote first-token
+ * latency (openai-hub.com/news/593, "华为云开源 KVarN：vLLM 原生 KV 缓存量化
+ * 后端", section 对开发者意味着什么: 180 -> 120 ms) but give no kernel for
+ * it; this is the decode path with (query, head) columns in place of heads.
  *
  *  q      fp16 [B][q_len][Hq][128]: query i of sequence b sits at position
  *         seq_len - q_len + i and attends keys [0, seq_len - q_len + i].
  *  out    fp16 [B][q_len][Hq][128].
- *  The q_len tokens' own K/V must already be in the cache (normally in the
- *  fp16 tail, e.g. by kvarn_decode_attention_append); seq_len counts them.
+ *  The q_len tokens' own K/V must already be in the cache -- in the fp16 tail
+ *  or, once a tile of 128 has filled, in the packed tile (which is then read
+ *  with a per-query causal mask); seq_len counts them.
  *  Other arguments as kvarn_decode_attention.
  *  workspace  at least kvarn_decode_multiquery_workspace_bytes(cfg, dims, q_len).
- * Requires 1 <= q_len <= KVARN_MAX_Q_LEN.  Every query must lie at or after the
- * final token of the last full tile, i.e. (seq_len mod 128) + 1 >= q_len and
- * seq_len >= q_len: then only the fp16 tail is masked.  A sequence that breaks
- * this is reported as KVARN_DEV_BAD_SEQ_LEN and its outputs are 0.  q_len = 1
- * is exactly kvarn_decode_attention. */
+ * Requires 1 <= q_len <= KVARN_MAX_Q_LEN and seq_len >= q_len; as q_len <= 128,
+ * the queries reach back at most into the last full tile.  A sequence with
+ * seq_len < q_len is reported as KVARN_DEV_BAD_SEQ_LEN and its outputs are 0.
+ * q_len = 1 is exactly kvarn_decode_attention. */
 KVARN_API size_t kvarn_decode_multiquery_workspace_bytes(const kvarn_config* cfg, const kvarn_decode_dims* dims,
                                                          int32_t q_len);
 
@@ -245,8 +250,11 @@ KVARN_API kvarn_status kvarn_decode_attention_multiquery(const void* q, int32_t 
  *    > KVARN_NOALLOC_SCRATCH_BYTES) the call returns
  *    KVARN_ERR_WORKSPACE_TOO_SMALL and launches nothing.
  *  - The first call on each device looks up the array's device address
- *    (cudaGetSymbolAddress) with that device current and caches it; make that
- *    first call before any stream capture begins.
+ *    (cudaGetSymbolAddress) with that device current and caches it for the
+ *    life of the process; make that first call before any stream capture
+ *    begins.  The cache is keyed by device ordinal: after the device's
+ *    primary context is reset (cudaDeviceReset) the cached address is stale,
+ *    so do not use this entry point across such a reset.
  *  - All calls on a device share the one array and it keeps the previous
  *    call's contents.  The only words that must start at zero are the
  *    per-(sequence, KV head) arrival counters, and each call clears them

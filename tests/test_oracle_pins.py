@@ -453,20 +453,71 @@ def test_multiquery_single_query_is_decode():
 
 
 def test_multiquery_query_i_is_decode_of_the_prefix_it_sees():
-    """Query i attends exactly the first L - qlen + i + 1 tokens: the plain
-    decode of a sequence cut to that length, over the same cache."""
+    """Query i attends exactly the first L - qlen + i + 1 tokens: where that
+    prefix ends in the fp16 tail or at the end of a full tile, it is the plain
+    decode of the sequence cut to that length, over the same cache."""
     qlen = 5
-    lens = [256 + 4, 128 + 100, 20, 128 + 3]          # the last one breaks the precondition (3 + 1 < 5)
+    lens = [256 + 4, 128 + 100, 20, 128 + 3, 2 * 128 + 2]
     w = inputs.make_decode_workload("mq", lens, 8, 2, seed=63, pool_blocks=8)
     packed, scales = O.quantize_tiles(w.k_full, w.v_full, w.slot_mapping, 2, w.num_blocks, 4, 2)
     q = np.random.default_rng(64).standard_normal((len(lens), qlen, 8, 128)).astype(np.float16)
     out = O.decode_multiquery(q, packed, scales, w.tail, w.block_table, w.seq_lens, 2, 4, 2)
+    checked = 0
     for i in range(qlen):
         cut = np.array([L - qlen + i + 1 for L in lens], dtype=np.int32)
         ref = O.decode(q[:, i], packed, scales, w.tail, w.block_table, cut, 2, 4, 2)
-        for b in range(3):
-            assert np.array_equal(out[b, i], ref[b])
-    assert np.all(out[3] == 0)
+        for b, L in enumerate(lens):
+            if cut[b] // 128 == L // 128:           # the prefix keeps every full tile
+                assert np.array_equal(out[b, i], ref[b])
+                checked += 1
+    # sequences 3 and 4: the queries before the tail sit in the last full
+    # tile; the one at its final token is the decode of exactly the full tiles
+    assert checked == 3 * qlen + 4 + 3
+    assert np.all(out[:, :, :, :].astype(np.float32).any(axis=-1))
+
+
+def test_multiquery_inside_a_packed_tile_is_causal():
+    """Queries whose position lies inside the last full tile (so that tile
+    must be masked per query): changing the stored codes of tokens after a
+    query's position, or the fp16 tail, leaves its output unchanged; changing
+    the codes of a token it sees changes it."""
+    qlen = 6
+    L = 3 * 128 + 2                                   # queries at 380..385: 380..383 in tile 2
+    w = inputs.make_decode_workload("mqc", [L], 4, 1, seed=65, pool_blocks=4)
+    packed, scales = O.quantize_tiles(w.k_full, w.v_full, w.slot_mapping, 1, w.num_blocks, 4, 2)
+    q = np.random.default_rng(66).standard_normal((1, qlen, 4, 128)).astype(np.float16)
+    base = O.decode_multiquery(q, packed, scales, w.tail, w.block_table, w.seq_lens, 1, 4, 2)
+    blk = int(w.block_table[0, 2])
+
+    def with_codes(edit):
+        """The cache with tile 2's K and V codes ([t][d]) passed through edit."""
+        p = packed.copy()
+        for side, bits, off in (("K", 4, 0), ("V", 2, O.side_bytes(4))):
+            n = O.side_bytes(bits)
+            c = O.unpack_codes(p[blk, 0, off:off + n], side, bits)
+            p[blk, 0, off:off + n] = O.pack_codes(edit(c, 2 ** bits - 1), side, bits)
+        return p
+
+    for i in range(4):                                # query i sits at tile-2 token 124 + i
+        t = 124 + i
+
+        def later(c, lb):
+            c = c.copy()
+            c[t + 1:] = lb - c[t + 1:]
+            return c
+
+        def own(c, lb):
+            c = c.copy()
+            c[t] = lb - c[t]
+            return c
+
+        t2 = w.tail.copy()
+        t2[0, :, 0, :2] = -t2[0, :, 0, :2]
+        got = O.decode_multiquery(q, with_codes(later), scales, t2, w.block_table, w.seq_lens, 1, 4, 2)
+        assert np.array_equal(got[0, i], base[0, i]), i
+        assert not np.array_equal(got[0, 4:], base[0, 4:])   # the tail queries see both changes
+        got3 = O.decode_multiquery(q, with_codes(own), scales, w.tail, w.block_table, w.seq_lens, 1, 4, 2)
+        assert not np.array_equal(got3[0, i], base[0, i]), i
 
 
 def test_append_steps_across_a_tile_fill():
