@@ -47,30 +47,56 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(f) <= t for f in _inputs())
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and up_to_date():
-        return LIB
-    objdir = os.path.join(HERE, "_build")
-    os.makedirs(objdir, exist_ok=True)
-    objs = []
-    for src in SOURCES:
-        obj = os.path.join(objdir, src.replace(".cu", ".o"))
-        cmd = [nvcc(), *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"), "-c", os.path.join(CSRC, src), "-o", obj]
-        r = subprocess.run(cmd, capture_output=True, text=True)
-        if r.returncode != 0:
-            sys.stderr.write(r.stdout + r.stderr)
-            raise RuntimeError(f"nvcc failed on {src}")
-        if verbose:
-            sys.stderr.write(r.stderr)
-        objs.append(obj)
-    tmp = LIB + ".tmp"
+# A test-only variant of the library: the decode's first copy of one warp
+# never arrives and the copy waits give up after 2^10 polls, so a test can
+# check that the kernel returns KVARN_DEV_TIMEOUT and leaves the device usable.
+STALL_LIB = os.path.join(HERE, "libkvarn_stalltest.so")
+STALL_DEFINES = ["-DKVARN_TEST_STALL_FIRST_UNIT=1", "-DKVARN_WAIT_LIMIT_LOG2=10"]
+
+
+def _compile(src: str, obj: str, defines, verbose: bool) -> None:
+    cmd = [nvcc(), *NVCC_FLAGS, *defines, "-I", os.path.join(ROOT, "include"), "-c", os.path.join(CSRC, src),
+           "-o", obj]
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    if r.returncode != 0:
+        sys.stderr.write(r.stdout + r.stderr)
+        raise RuntimeError(f"nvcc failed on {src}")
+    if verbose:
+        sys.stderr.write(r.stderr)
+
+
+def _link(objs, lib: str) -> None:
+    tmp = lib + ".tmp"
     cmd = [nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-Xcompiler", "-fPIC",
            "-o", tmp, *objs]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         sys.stderr.write(r.stdout + r.stderr)
         raise RuntimeError("link failed")
-    os.replace(tmp, LIB)
+    os.replace(tmp, lib)
+
+
+def _fresh(lib: str) -> bool:
+    if not os.path.exists(lib):
+        return False
+    t = os.path.getmtime(lib)
+    return all(os.path.getmtime(f) <= t for f in _inputs())
+
+
+def build(force: bool = False, verbose: bool = False) -> str:
+    if not force and up_to_date() and _fresh(STALL_LIB):
+        return LIB
+    objdir = os.path.join(HERE, "_build")
+    os.makedirs(objdir, exist_ok=True)
+    objs = []
+    for src in SOURCES:
+        obj = os.path.join(objdir, src.replace(".cu", ".o"))
+        _compile(src, obj, [], verbose)
+        objs.append(obj)
+    _link(objs, LIB)
+    stall_obj = os.path.join(objdir, "decode_stalltest.o")
+    _compile("decode.cu", stall_obj, STALL_DEFINES, verbose)
+    _link([stall_obj if o.endswith(os.sep + "decode.o") else o for o in objs], STALL_LIB)
     return LIB
 
 

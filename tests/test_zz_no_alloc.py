@@ -1,7 +1,8 @@
 """The allocation-free decode entry point (kvarn_decode_attention_noalloc).
 
-It is for callers that cannot allocate device memory themselves; its
-split-K scratch is a fixed device array inside the library.  Here it is
+It is for callers that cannot allocate device memory themselves; the
+partial-record scratch of its stream-K decode is a fixed device array inside
+the library.  Here it is
 called straight through the C ABI and its output is checked against the
 workspace-taking kvarn_decode_attention on the same inputs, within the
 decode tolerance the parity tests use, on two calls in a row (the second
@@ -74,7 +75,8 @@ def test_noalloc_matches_workspace_entry_point_twice(K):
 
 def test_noalloc_rejects_problems_beyond_its_scratch(K):
     cfg = K.config("kvarn_k4v2_g128")
-    # B * Hq * (splits + 1) partial records of 528 B exceed the fixed 8 MiB array
+    # (B*Hkv + 320)*G tile records plus B*Hkv*G tail records of 528 B (and the
+    # counters) exceed the fixed 8 MiB array
     d = K.dims(4096, 64, 8, 64, 4096)
     assert K.decode_workspace_bytes(cfg, d) > (8 << 20)
     one = torch.zeros(16, dtype=torch.uint8, device="cuda")
