@@ -15,8 +15,8 @@ Per-kernel CUDA-event times give the quantise tiles/s, the decode-only
 tokens/s and each kernel's HBM GB/s from algorithmic bytes.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
---impl reference times the CPU oracle (the fp64 restatement in oracle/) on a
-bounded sample of the same step, extrapolated to the full step.
+--impl reference times the CPU oracle (the fp64 restatement in oracle/) on
+whole steps of the same workload, spread over all of the host's cores.
 """
 from __future__ import annotations
 
@@ -58,7 +58,7 @@ def load_peaks():
 # ------------------------------------------------------------------ clocks (NVML, sampled in a thread)
 
 class ClockSampler:
-    def __init__(self, device_index: int, period_s: float = 0.005):
+    def __init__(self, device_index: int, period_s: float = 0.0005):
         self.samples, self.reasons = [], set()
         self.max_mhz = None
         self._stop = threading.Event()
@@ -161,6 +161,13 @@ def run_gpu(args):
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    w, rows = build_workload(rank)
+    oracle_step = None
+    if world == 1 and not args.no_cpu_baseline:
+        # the CPU baseline's worker pool is forked now, before this process
+        # first touches the GPU
+        from oracle.parallel_step import OracleStep
+        oracle_step = OracleStep(w, rows)
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if world > 1:
@@ -169,7 +176,6 @@ def run_gpu(args):
 
     from bit_kv_cache_15_b200 import kvarn as K
 
-    w, rows = build_workload(rank)
     cfg = K.config("kvarn_k4v2_g128")
     packed, scales = K.alloc_cache(cfg, w.num_blocks, HKV, device=dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
@@ -306,7 +312,7 @@ def run_gpu(args):
             "higher_is_better": True,
             "scaling": "weak",
             "vs_baseline": None,
-            "dtype": "fp16 in/out, k4v2 codes, fp32 accumulate",
+            "dtype": "f32 (fp16 in/out, k4v2 codes, fp32 arithmetic and accumulation)",
             "data": "synthetic (seeded; Llama/Qwen-shaped GQA, outlier channels + lognormal token scales)",
             "config": {"workload": WORKLOAD, "global_batch": BATCH * world, "seq_len": 16384,
                        "parallelism": f"data-parallel x{world}: each rank its own 8 sequences, no collective on the path",
@@ -330,10 +336,12 @@ def run_gpu(args):
         }
         if world == 1 and not args.no_sweep:
             line["sweep"] = {"workload": "decode only, batch 8 at 16384 + ragged tail, Hq=64 Hkv=8, L2 flushed "
-                                         "before each call", "results": precision_sweep(w, dev)}
-        if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline(w, rows, budget_s=args.cpu_budget)
+                                         "before each call", "results": precision_sweep(w, rows, dev)}
+        if oracle_step is not None:
+            line["cpu_baseline"] = cpu_baseline(oracle_step)
         print(json.dumps(line), flush=True)
+    if oracle_step is not None:
+        oracle_step.close()
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -341,11 +349,13 @@ def run_gpu(args):
 
 # ------------------------------------------------------------------ precision sweep (outside the timed step)
 
-def precision_sweep(w, dev, iters=30):
+def precision_sweep(w, rows, dev, iters=30):
     """Decode-only time of the same batch-8 16K (+tail) problem at k8v8 / k4v4 /
     k4v2 / k2v2 and over uncompressed fp16 and e4m3 caches (the in-library
-    baselines).  Each call is timed alone with CUDA events after a 256 MB write
-    that flushes L2.  Returns {name: {us, tokens_per_s, hbm_gbs, bytes}}."""
+    baselines); the quantiser on the step's 4096 appended tiles at each width;
+    and the k4v2 decode of the Llama-3-8B- and Llama-3-70B-shaped workloads.
+    Each call is timed alone with CUDA events after a 256 MB write that
+    flushes L2.  Returns {name: {us, ...}}."""
     import torch
     from bit_kv_cache_15_b200 import kvarn as K
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
@@ -376,10 +386,19 @@ def precision_sweep(w, dev, iters=30):
     kf = torch.from_numpy(w.k_full).to(dev)
     vf = torch.from_numpy(w.v_full).to(dev)
     slot = torch.from_numpy(w.slot_mapping).to(dev)
+    k_app, v_app, slot_app = kf[rows], vf[rows], slot[rows]
+    tiles = len(rows) // 128 * HKV * 2
+    hbm_peak, _ = load_peaks()
     for kb, vb in ((8, 8), (4, 4), (4, 2), (2, 2)):
         cfg = K.config(f"kvarn_k{kb}v{vb}_g128")
         packed, scales = K.alloc_cache(cfg, w.num_blocks, HKV, device=dev)
         K.quantize_tiles(kf, vf, slot, packed, scales, cfg)
+        us = timed(lambda: K.quantize_tiles(k_app, v_app, slot_app, packed, scales, cfg))
+        qbytes = len(rows) // 128 * HKV * (2 * 32768 + 2048 * (kb + vb) + 2 * 528 + 16)
+        res[f"quantize_k{kb}v{vb}"] = {"us": us, "tiles_per_s": tiles / (us * 1e-6), "tiles": tiles,
+                                        "hbm_gbs": qbytes / (us * 1e-6) / 1e9,
+                                        "frac_of_measured_hbm": qbytes / (us * 1e-6) / 1e9 / hbm_peak,
+                                        "tflops": tiles * QUANT_FLOPS_PER_TILE / (us * 1e-6) / 1e12}
         d = K.dims(BATCH, HQ, HKV, w.max_blocks_per_seq, w.num_blocks)
         ws = torch.empty(K.decode_workspace_bytes(cfg, d), dtype=torch.uint8, device=dev)
         us = timed(lambda: K.decode_attention(q, packed, scales, tail, bt, sl, cfg, out=out, workspace=ws))
@@ -417,6 +436,43 @@ def precision_sweep(w, dev, iters=30):
     us = timed(lambda: K.decode_attention_fp8(q, k8, v8, bt2d, sl, k_scale, v_scale, out=out, workspace=wsb))
     nbytes = HKV * (n_full_tok + tail_tok) * 256 + 2 * BATCH * HQ * 256
     res["fp8"] = {"us": us, "tokens_per_s": BATCH / (us * 1e-6), "hbm_gbs": nbytes / (us * 1e-6) / 1e9, "bytes": nbytes}
+    del k8, v8, wsb
+    res.update(config_decodes(dev, timed))
+    return res
+
+
+def config_decodes(dev, timed):
+    """k4v2 decode of the Llama-3-8B-shaped (B=16 x 4096, 32/8 heads) and the
+    Llama-3-70B-shaped (B=4, lengths U[1024, 131072], 64/8 heads) workloads,
+    each cache quantised first, the decode timed alone."""
+    import torch
+    from bit_kv_cache_15_b200 import inputs
+    from bit_kv_cache_15_b200 import kvarn as K
+    hbm_peak, kind = load_peaks()
+    res = {}
+    for name, make in (("llama3_8b_b16_4k", inputs.llama3_8b), ("llama3_70b_b4_1k_128k", inputs.llama3_70b)):
+        w = make()
+        cfg = K.config("kvarn_k4v2_g128")
+        packed, scales = K.alloc_cache(cfg, w.num_blocks, w.num_kv_heads, device=dev)
+        K.quantize_tiles(torch.from_numpy(w.k_full).to(dev), torch.from_numpy(w.v_full).to(dev),
+                         torch.from_numpy(w.slot_mapping).to(dev), packed, scales, cfg)
+        q = torch.from_numpy(w.q).to(dev)
+        tail = torch.from_numpy(w.tail).to(dev)
+        bt = torch.from_numpy(w.block_table).to(dev)
+        sl = torch.from_numpy(w.seq_lens).to(dev)
+        out = torch.empty_like(q)
+        d = K.dims(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.max_blocks_per_seq, w.num_blocks)
+        ws = torch.empty(K.decode_workspace_bytes(cfg, d), dtype=torch.uint8, device=dev)
+        us = timed(lambda: K.decode_attention(q, packed, scales, tail, bt, sl, cfg, out=out, workspace=ws))
+        lens = [int(x) for x in w.seq_lens]
+        nbytes = (w.num_kv_heads * sum(L // 128 * (12288 + 1056 + 4) + L % 128 * 512 for L in lens)
+                  + 2 * w.num_seqs * w.num_q_heads * 256)
+        gbs = nbytes / (us * 1e-6) / 1e9
+        res[name] = {"us": us, "tokens_per_s": w.num_seqs / (us * 1e-6),
+                     "context_tokens_per_s": sum(lens) / (us * 1e-6), "seq_lens": lens, "bytes": nbytes,
+                     "hbm_gbs": gbs, "frac_of_measured_hbm": gbs / hbm_peak, "frac_of_8tbs": gbs / 8000.0}
+        del packed, scales, w
+        torch.cuda.empty_cache()
     return res
 
 
@@ -484,90 +540,45 @@ def append_step(w, dev, cfg, kf, vf, slot, q, tail, sl, out, ws, decode_bytes, t
 
 # ------------------------------------------------------------------ the oracle (CPU baseline / reference arm)
 
-def oracle_step_sample(w, rows, n_tiles, n_pairs, seed=0):
-    """Time the oracle on n_tiles of the append batch and n_pairs (seq, KV head)
-    decodes (all G query heads), extrapolated to one full step."""
-    from oracle import kvarn_oracle as O
-    rng = np.random.default_rng(seed)
-    groups = len(rows) // 128
-    k_app, v_app = w.k_full[rows], w.v_full[rows]
-    t0 = time.perf_counter()
-    for _ in range(n_tiles):
-        g = int(rng.integers(groups))
-        h = int(rng.integers(HKV))
-        side = int(rng.integers(2))
-        src = k_app if side == 0 else v_app
-        O.quantize_tile(np.ascontiguousarray(src[g * 128:(g + 1) * 128, h]), 4 if side == 0 else 2, 8)
-    tq = time.perf_counter() - t0
-    # a small paged cache holding just the sampled pairs' tiles, quantised by the oracle (untimed)
-    G = HQ // HKV
-    t_dec = 0.0
-    for _ in range(n_pairs):
-        b = int(rng.integers(BATCH))
-        h = int(rng.integers(HKV))
-        s, e = w.token_range(b)
-        n_full = (e - s) // 128
-        sub_k = w.k_full[s:e, h:h + 1]
-        sub_v = w.v_full[s:e, h:h + 1]
-        slot = np.arange(e - s, dtype=np.int64)
-        packed, scales = O.quantize_tiles(sub_k, sub_v, slot, 1, n_full, 4, 2)
-        bt = np.arange(n_full, dtype=np.int32)[None, :]
-        q = w.q[b:b + 1, h * G:(h + 1) * G]
-        tail = w.tail[b:b + 1, :, h:h + 1]
-        t1 = time.perf_counter()
-        O.decode(q, packed, scales, tail, bt, w.seq_lens[b:b + 1], 1, 4, 2)
-        t_dec += time.perf_counter() - t1
-    tiles_total = groups * HKV * 2
-    pairs_total = BATCH * HKV
-    t_step = tq * tiles_total / max(n_tiles, 1) + t_dec * pairs_total / max(n_pairs, 1)
-    return t_step, tq + t_dec
+ORACLE_STEP = ("one whole step of the same workload: the oracle (numpy fp64) quantises the 4096 appended K+V "
+               "tiles into the paged cache, then decodes all 64 (sequence, KV head) pairs; one process per host "
+               "core, one BLAS thread each; the rest of the cache is quantised once before timing")
 
 
-def _blas_threads():
-    try:
-        from threadpoolctl import threadpool_info
-        return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
-    except Exception:
-        return 1
-
-
-def cpu_baseline(w, rows, budget_s=20.0):
-    from threadpoolctl import threadpool_limits
-    with threadpool_limits(1):
-        t_step, spent = oracle_step_sample(w, rows, n_tiles=256, n_pairs=2)
-        reps = max(1, int(budget_s / max(spent, 1e-3)) - 1)
-        if reps > 1:
-            t_step2, spent2 = oracle_step_sample(w, rows, n_tiles=256 * reps, n_pairs=min(2 * reps, BATCH * HKV), seed=1)
-            t_step, spent = t_step2, spent + spent2
-    return {"value": BATCH / t_step, "unit": "decode tokens/s", "cores": 1, "kind": "oracle",
-            "sample": f"oracle (numpy fp64, 1 thread) on sampled append tiles and (seq, KV head) decodes of the "
-                      f"same step, extrapolated to 4096 tiles + 64 pairs; {spent:.1f} s of CPU work"}
+def cpu_baseline(oracle_step, steps=1):
+    """The oracle timed on whole steps over all host cores (no extrapolation)."""
+    oracle_step.prefill()
+    ts = oracle_step.timed_steps(steps)
+    t = statistics.median(ts)
+    return {"value": BATCH / t, "unit": "decode tokens/s", "cores": oracle_step.workers, "kind": "oracle",
+            "sample": f"{ORACLE_STEP}; {steps} step(s), {t:.2f} s each"}
 
 
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    from threadpoolctl import threadpool_limits
+    from oracle.parallel_step import OracleStep
     w, rows = build_workload()
-    with threadpool_limits(1):
-        for i in range(args.warmup):
-            oracle_step_sample(w, rows, n_tiles=16, n_pairs=1, seed=100 + i)
-        t_steps, spent = [], 0.0
-        for i in range(args.steps):
-            t_step, s = oracle_step_sample(w, rows, n_tiles=32, n_pairs=1, seed=i)
-            t_steps.append(t_step)
-            spent += s
-    t_mean = float(np.mean(t_steps))
+    st = OracleStep(w, rows)
+    try:
+        st.prefill()
+        st.timed_steps(args.warmup)
+        t_steps = st.timed_steps(args.steps)
+    finally:
+        st.close()
+    total = float(np.sum(t_steps))
+    t_mean = total / len(t_steps)
     value = BATCH / t_mean
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "decode tokens/s", "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_mean * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)", "data": "synthetic (seeded)",
-        "config": {"workload": WORKLOAD, "global_batch": BATCH, "seq_len": 16384, "parallelism": "none (CPU)"},
-        "cpu_baseline": {"value": value, "unit": "decode tokens/s", "cores": 1, "kind": "oracle",
-                         "sample": f"each step: 32 sampled append tiles + 1 (seq, KV head) decode, extrapolated to "
-                                   f"the full step; {spent:.1f} s of CPU work in total"},
+        "config": {"workload": WORKLOAD, "global_batch": BATCH, "seq_len": 16384,
+                   "parallelism": f"none (CPU: {st.workers} worker processes)"},
+        "cpu_baseline": {"value": value, "unit": "decode tokens/s", "cores": st.workers, "kind": "oracle",
+                         "sample": f"{ORACLE_STEP}; {args.steps} timed steps after {args.warmup} warm-up steps, "
+                                   f"{total:.1f} s timed in total"},
         "e2e": {"value": value, "unit": "decode tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -579,7 +590,6 @@ def main():
     ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sweep", action="store_true")
     args = ap.parse_args()
