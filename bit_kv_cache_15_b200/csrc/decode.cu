@@ -830,11 +830,14 @@ __device__ __forceinline__ bool decode_segment(const DecodeArgs& p, uint8_t* sme
 // kTailUnits for the fp16 tail (which also carries an empty or invalid
 // sequence, so every pair is owned).  The tail, and usually the merge of the
 // pair, fall to the CTA owning the pair's last unit; weighting them as
-// several tiles keeps that CTA's range shorter.
+// several tiles keeps that CTA's range shorter.  A pair with no tail rows
+// (seq_len a multiple of 128, nothing appended) weighs kTailUnitsEmpty: the
+// merge and a segment restart only.
 // A tail that an appended token fills is also quantised, K and V as two more
 // work items of kFillUnits each after the tail (rotation recomputed), so that
 // up to three CTAs share a fill.  Each item falls to the CTA holding its last unit.
 constexpr int kTailUnits = 9;
+constexpr int kTailUnitsEmpty = 3;
 constexpr int kFillUnits = 16;
 
 // With qlen > 1 the sequence must hold its qlen query tokens (L >= qlen); as
@@ -843,9 +846,12 @@ __device__ __forceinline__ bool seq_valid(const DecodeArgs& p, int L) {
   return L >= 0 && L + p.append <= kTile * p.max_blocks && (p.qlen == 1 || L >= p.qlen);
 }
 __device__ __forceinline__ int pair_tiles(int L, bool valid) { return valid ? (L >> 7) : 0; }
+__device__ __forceinline__ int tail_units(const DecodeArgs& p, int L, bool valid) {
+  return valid && (L & 127) + p.append == 0 ? kTailUnitsEmpty : kTailUnits;
+}
 __device__ __forceinline__ int pair_units(const DecodeArgs& p, int L, bool valid) {
   const bool fills = valid && p.append && (L & 127) == kTile - 1;
-  return pair_tiles(L, valid) + kTailUnits + (fills ? 2 * kFillUnits : 0);
+  return pair_tiles(L, valid) + tail_units(p, L, valid) + (fills ? 2 * kFillUnits : 0);
 }
 
 // CTA i of P owns units [W*i/P, W*(i+1)/P); owner(u) inverts that.
@@ -1079,8 +1085,9 @@ __global__ void __launch_bounds__(kDThreads, KVARN_D_MIN_CTAS) decode_kernel(con
         sg_te = static_cast<int>(min(e - pst, static_cast<long long>(pair_tiles(L, seq_valid(p, L)))));
         // last units of the work items after the tiles: tail attention, then
         // (a filling append) quantise K, quantise V
-        const long long m_att = pst + pair_tiles(L, seq_valid(p, L)) + kTailUnits - 1;
-        const int items = nu - pair_tiles(L, seq_valid(p, L)) > kTailUnits ? 3 : 1;
+        const int tu = tail_units(p, L, seq_valid(p, L));
+        const long long m_att = pst + pair_tiles(L, seq_valid(p, L)) + tu - 1;
+        const int items = nu - pair_tiles(L, seq_valid(p, L)) > tu ? 3 : 1;
         int flags = 0;
 #pragma unroll
         for (int k = 0; k < 3; ++k) {

@@ -221,9 +221,10 @@ KVARN_API kvarn_status kvarn_decode_attention_append(const void* q, const void* 
  *  Other arguments as kvarn_decode_attention.
  *  workspace  at least kvarn_decode_multiquery_workspace_bytes(cfg, dims, q_len).
  * Requires 1 <= q_len <= KVARN_MAX_Q_LEN and seq_len >= q_len; as q_len <= 128,
- * the queries reach back at most into the last full tile.  A sequence with
- * seq_len < q_len is reported as KVARN_DEV_BAD_SEQ_LEN and its outputs are 0.
- * q_len = 1 is exactly kvarn_decode_attention. */
+ * the queries reach back at most into the last full tile.  With q_len > 1 a
+ * sequence with seq_len < q_len is reported as KVARN_DEV_BAD_SEQ_LEN and its
+ * outputs are 0.  q_len = 1 is exactly kvarn_decode_attention (an empty
+ * sequence gives 0 and no status). */
 KVARN_API size_t kvarn_decode_multiquery_workspace_bytes(const kvarn_config* cfg, const kvarn_decode_dims* dims,
                                                          int32_t q_len);
 

@@ -34,7 +34,8 @@ def libs():
 
 def test_decode_wait_timeout_is_reported_and_device_stays_usable(libs):
     K, stall = libs
-    w = inputs.make_decode_workload("timeout", [20 * 128 + 9, 6 * 128, 300], 16, 2, seed=990, pool_blocks=30)
+    # more work units than decode CTAs, so that CTA 0 (whose first copy stalls) has a range
+    w = inputs.make_decode_workload("timeout", [150 * 128 + 9, 60 * 128, 300], 16, 2, seed=990, pool_blocks=220)
     cfg = K.config()
     dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
     packed, scales = K.alloc_cache(cfg, w.num_blocks, 2)
