@@ -68,7 +68,10 @@ struct DecodeTraits {
   static constexpr int kQrotOff = kBarOff + 128;
   static constexpr int kScrOff = kQrotOff + kMaxG * kHeadDim * 4;
   static constexpr int kInvSigOff = kScrOff + kDWarps * kHeadDim * 4;
-  static constexpr int kSmem = kInvSigOff + 64;
+  // per-warp token-scale scratch of 1 KB: inside the q H buffer (free once every
+  // warp holds q H in registers), or its own area when q H is read per tile
+  static constexpr int kTokOff = kInvSigOff + 64;
+  static constexpr int kSmem = kTokOff + (KVARN_D_QR_SMEM ? kDWarps * 1024 : 0);
   static_assert(kStage % 16 == 0, "stage must stay 16-byte aligned");
   static_assert(kSmem <= 227 * 1024, "shared memory");
   static_assert(kDWarps * kDStages * 8 <= 128, "barrier area");
@@ -490,6 +493,12 @@ __device__ __forceinline__ bool decode_segment(const DecodeArgs& p, uint8_t* sme
       if (col_row(p, b, h, grp, 2 * c + j, &row, &qi)) climit[j] = L - p.qlen + qi - kTile * mask_tile;
     }
   }
+#if !KVARN_D_QR_SMEM
+  __syncthreads();   // every warp holds its q H: the q H buffer now serves as per-warp token-scale scratch
+  float* tokbuf = qrot + warp * 256;   // [2 (K, V)][8 (g8)][16 (mt, ri)]
+#else
+  float* tokbuf = reinterpret_cast<float*>(smem + T::kTokOff) + warp * 256;
+#endif
   const float coef0 = p.sm_scale * kLog2e * (1.f / 128.f) * invsig[2 * c];
   const float coef1 = p.sm_scale * kLog2e * (1.f / 128.f) * invsig[2 * c + 1];
   float* scr = reinterpret_cast<float*>(smem + T::kScrOff) + warp * kHeadDim;
@@ -539,6 +548,35 @@ __device__ __forceinline__ bool decode_segment(const DecodeArgs& p, uint8_t* sme
       const float zv = *reinterpret_cast<const float*>(rk + kScaleRec + 512);
       const float sv = *reinterpret_cast<const float*>(rk + kScaleRec + 516);
       const int t0 = part * (16 * MT);   // first token of this unit within the tile
+      // token scales once per token (MT / 2 tokens per lane): 2^Lt_k, and the V
+      // scales relative to the unit's largest, times 2^kPBoost (the weights
+      // p * tv fed to the V-side mma then stay in fp16's normal range down to
+      // p * tv ~ 2^-26 of the unit maximum; the factor is undone in the fold);
+      // read back below in the score layout
+      float lvm;
+      {
+        constexpr int TPL = MT / 2;
+        float lk[TPL], lv[TPL];
+#pragma unroll
+        for (int i = 0; i < TPL; ++i) {
+          lk[i] = hf(ltk, t0 + TPL * lane + i);
+          lv[i] = hf(ltv, t0 + TPL * lane + i);
+        }
+        float m = lv[0];
+#pragma unroll
+        for (int i = 1; i < TPL; ++i) m = fmaxf(m, lv[i]);
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        lvm = ceilf(m);
+#pragma unroll
+        for (int i = 0; i < TPL; ++i) {
+          const int tr = TPL * lane + i;   // token tr sits at lane g8 = tr % 8, slot (tr / 16, tr / 8 % 2)
+          const int idx = (tr & 7) * 16 + (tr >> 4) * 2 + ((tr >> 3) & 1);
+          tokbuf[idx] = ex2_fast(lk[i]);
+          tokbuf[128 + idx] = ex2_fast(lv[i] - lvm + static_cast<float>(kPBoost));
+        }
+        __syncwarp();
+      }
 
       // a6: channel scales with a power-of-two prescale so q' <= 1 in magnitude
       float lcl[4];
@@ -625,16 +663,21 @@ __device__ __forceinline__ bool decode_segment(const DecodeArgs& p, uint8_t* sme
       // the step with the codes' 2^(s - 24) placement undone, per row half
       constexpr float kRowK0 = 16777216.f / static_cast<float>(1 << CodeShift<KB>::kBase);
       constexpr float kRowK1 = kRowK0 / static_cast<float>(1 << CodeShift<KB>::kSRow);
-      float tv[MT][2];
+      float tv[MT][2], tkv[MT][2];
+#pragma unroll
+      for (int k4 = 0; k4 < MT / 2; ++k4) {
+        const float4 a = *reinterpret_cast<const float4*>(&tokbuf[g8 * 16 + 4 * k4]);
+        const float4 b = *reinterpret_cast<const float4*>(&tokbuf[128 + g8 * 16 + 4 * k4]);
+        tkv[2 * k4][0] = a.x; tkv[2 * k4][1] = a.y; tkv[2 * k4 + 1][0] = a.z; tkv[2 * k4 + 1][1] = a.w;
+        tv[2 * k4][0] = b.x; tv[2 * k4][1] = b.y; tv[2 * k4 + 1][0] = b.z; tv[2 * k4 + 1][1] = b.w;
+      }
       float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
         for (int ri = 0; ri < 2; ++ri) {
-          const int t = t0 + 16 * mt + g8 + 8 * ri;
-          const float tk = ex2_fast(hf(ltk, t));
+          const float tk = tkv[mt][ri];
           const float skr = sk * (ri ? kRowK1 : kRowK0);
-          tv[mt][ri] = hf(ltv, t);
           S[mt][2 * ri] = fmaf(skr, S[mt][2 * ri], za0) * (cf0 * tk);
           S[mt][2 * ri + 1] = fmaf(skr, S[mt][2 * ri + 1], za1) * (cf1 * tk);
           mx0 = fmaxf(mx0, S[mt][2 * ri]);
@@ -664,20 +707,6 @@ __device__ __forceinline__ bool decode_segment(const DecodeArgs& p, uint8_t* sme
           mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
         }
       }
-      // V token scales relative to the tile's largest, times 2^kPBoost: the weights
-      // p * tv fed to the mma then stay in fp16's normal range down to p * tv ~ 2^-26
-      // of the tile maximum; the common factor is undone on the fold below
-      float lvm = tv[0][0];
-#pragma unroll
-      for (int mt = 0; mt < MT; ++mt) lvm = fmaxf(lvm, fmaxf(tv[mt][0], tv[mt][1]));
-      lvm = fmaxf(lvm, __shfl_xor_sync(0xffffffffu, lvm, 4));
-      lvm = fmaxf(lvm, __shfl_xor_sync(0xffffffffu, lvm, 8));
-      lvm = fmaxf(lvm, __shfl_xor_sync(0xffffffffu, lvm, 16));
-      lvm = ceilf(lvm);
-#pragma unroll
-      for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-        for (int ri = 0; ri < 2; ++ri) tv[mt][ri] = ex2_fast(tv[mt][ri] - lvm + static_cast<float>(kPBoost));
       const float mn0 = fmaxf(mrun[0], mx0), mn1 = fmaxf(mrun[1], mx1);
       // a column that has attended no token yet (masked) keeps max -inf: its
       // exponents are taken against 0, so its weights are 0 instead of NaN

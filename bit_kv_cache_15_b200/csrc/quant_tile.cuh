@@ -12,7 +12,8 @@
 //             warp reduce-scatter and (for channels) a 4-warp shared sum;
 //   4 quantise   Z = (R * fp32(2^-Lt)) * fp32(2^-Lc) from the stored fp16
 //             log-scales, one zero/step per tile from min/max, codes =
-//             clamp(rne((Z - zero) * (1/step)));
+//             clamp(rne((Z - zero) / step)), the quotient formed in fp32 as
+//             Z * (1/step) - zero * (1/step) (one FMA per element);
 //   5 pack    codes in the decode's mma fragment order, 16-byte stores.
 // The K-side rotation uses X as the mma A operand and the V side as the B
 // operand, so after stage 2 each lane holds exactly the elements of the
@@ -32,7 +33,8 @@ constexpr int kBox = 128 * 128;       // one 64-channel box: 128 rows of 128 byt
 // Per-CTA scratch of one tile's normalisation and quantisation.
 struct QuantScratch {
   float red[4][kHeadDim];                // per-warp channel partial sums
-  float u[kHeadDim];                     // channel weights 2^(-2 lc)
+  alignas(16) float u[kHeadDim];         // channel weights 2^(-2 lc), channel 16a + g + 8ri at g*16 + 2a + ri
+  alignas(16) float wb[4][32];           // per-warp token-weight exchange
   float mt[kTile];                       // fp32(2^-Lt)
   float mc[kHeadDim];                    // fp32(2^-Lc)
   float zmin[4], zmax[4];
@@ -368,7 +370,7 @@ __device__ __forceinline__ void quantize_tile(const TileOut& o, QuantScratch& sm
     {
       const float tot = (sm.red[0][tid] + sm.red[1][tid]) + (sm.red[2][tid] + sm.red[3][tid]);
       lc_sum = tot;
-      sm.u[tid] = weight_of_sum(tot);
+      sm.u[KL ? tid : (tid & 7) * 16 + (tid >> 4) * 2 + ((tid >> 3) & 1)] = weight_of_sum(tot);
     }
     __syncthreads();
 
@@ -406,9 +408,10 @@ __device__ __forceinline__ void quantize_tile(const TileOut& o, QuantScratch& sm
     } else {
       float uu[16];
 #pragma unroll
-      for (int a = 0; a < 8; ++a)
-#pragma unroll
-        for (int ri = 0; ri < 2; ++ri) uu[a * 2 + ri] = sm.u[16 * a + g + 8 * ri];
+      for (int k4 = 0; k4 < 4; ++k4) {
+        const float4 x = *reinterpret_cast<const float4*>(&sm.u[g * 16 + 4 * k4]);
+        uu[4 * k4] = x.x; uu[4 * k4 + 1] = x.y; uu[4 * k4 + 2] = x.z; uu[4 * k4 + 3] = x.w;
+      }
       float s[8];    // index ntl*2 + rj
 #pragma unroll
       for (int ntl = 0; ntl < 4; ++ntl) {
@@ -429,9 +432,13 @@ __device__ __forceinline__ void quantize_tile(const TileOut& o, QuantScratch& sm
       rs_step<4>(s, 8, lane);
       rs_step<2>(s, 4, lane);
       lt_sum = s[0];
-      const float wown = weight_of_sum(s[0]);
-#pragma unroll
-      for (int k = 0; k < 8; ++k) wt[k] = __shfl_sync(0xffffffffu, wown, c | (k << 2));
+      sm.wb[warp][c * 8 + g] = weight_of_sum(s[0]);
+      __syncwarp();
+      const float4 w0 = *reinterpret_cast<const float4*>(&sm.wb[warp][c * 8]);
+      const float4 w1 = *reinterpret_cast<const float4*>(&sm.wb[warp][c * 8 + 4]);
+      wt[0] = w0.x; wt[1] = w0.y; wt[2] = w0.z; wt[3] = w0.w;
+      wt[4] = w1.x; wt[5] = w1.y; wt[6] = w1.z; wt[7] = w1.w;
+      __syncwarp();
     }
   }
 
@@ -518,6 +525,7 @@ __device__ __forceinline__ void quantize_tile(const TileOut& o, QuantScratch& sm
   float step = __fdiv_rn(__fsub_rn(zmx, zero), static_cast<float>(LB));
   if (step == 0.f) step = 1.f;
   const float inv = __fdiv_rn(1.f, step);
+  const float nzi = -zero * inv;
 
   // codes: y = (Z - zero) * inv >= 0, rounded to nearest even by adding 1.5 * 2^23
   // (exact for y < 2^22); packed in the fragment order (block bl, register j, half h)
@@ -539,7 +547,7 @@ __device__ __forceinline__ void quantize_tile(const TileOut& o, QuantScratch& sm
         const int ntl = 2 * (bl >> 3) + (j >> 1), a = bl & 7, ri = j & 1;
         idx = (ntl * 8 + a) * 4 + 2 * ri;
       }
-      const float2 y = __fmul2_rn(__fadd2_rn(f2(Z[idx], Z[idx + 1]), f2(-zero, -zero)), f2(inv, inv));
+      const float2 y = __ffma2_rn(f2(Z[idx], Z[idx + 1]), f2(inv, inv), f2(nzi, nzi));
       const float2 r = __fadd2_rn(y, f2(kMagic, kMagic));
       // 0 <= y <= 2^b - 1 up to rounding, so rne(y) sits in the low BITS bits of r
       if (SIDE == 0 && !KL) {

@@ -131,8 +131,8 @@ KVARN_API size_t kvarn_decode_workspace_bytes(const kvarn_config* cfg, const kva
  * Each (group, head, K|V) tile: R = X H (Sylvester Hadamard, unnormalised);
  * sinkhorn_iters passes of channel then token RMS normalisation in base-2 log
  * space; log-scales stored fp16; Z = (R*2^-Lt)*2^-Lc in fp32; one zero/step
- * per tile from min/max; codes = clamp(rne((Z-zero)*(1/step))) packed in the
- * mma-fragment order.  Groups whose slot is invalid are skipped and reported
+ * per tile from min/max; codes = clamp(rne((Z-zero)/step)), the quotient taken
+ * in fp32 as Z*(1/step) - zero*(1/step), packed in the mma-fragment order.  Groups whose slot is invalid are skipped and reported
  * as KVARN_DEV_BAD_SLOT. */
 KVARN_API kvarn_status kvarn_quantize_tiles(const void* k, const void* v, const int64_t* slot_mapping,
                                   int64_t num_tokens, int32_t num_kv_heads, int64_t num_blocks,
