@@ -43,9 +43,6 @@ namespace {
 #ifndef KVARN_D_MIN_CTAS
 #define KVARN_D_MIN_CTAS 2
 #endif
-#ifndef KVARN_D_QR_SMEM
-#define KVARN_D_QR_SMEM 0      // 1: read q H from shared memory per tile instead of holding it in registers
-#endif
 
 constexpr int kDWarps = 4;
 constexpr int kDThreads = 32 * kDWarps;
@@ -68,10 +65,9 @@ struct DecodeTraits {
   static constexpr int kQrotOff = kBarOff + 128;
   static constexpr int kScrOff = kQrotOff + kMaxG * kHeadDim * 4;
   static constexpr int kInvSigOff = kScrOff + kDWarps * kHeadDim * 4;
-  // per-warp token-scale scratch of 1 KB: inside the q H buffer (free once every
-  // warp holds q H in registers), or its own area when q H is read per tile
-  static constexpr int kTokOff = kInvSigOff + 64;
-  static constexpr int kSmem = kTokOff + (KVARN_D_QR_SMEM ? kDWarps * 1024 : 0);
+  // the per-warp token-scale scratch (1 KB) sits inside the q H buffer, which
+  // is free once every warp holds q H in registers
+  static constexpr int kSmem = kInvSigOff + 64;
   static_assert(kStage % 16 == 0, "stage must stay 16-byte aligned");
   static_assert(kSmem <= 227 * 1024, "shared memory");
   static_assert(kDWarps * kDStages * 8 <= 128, "barrier area");
@@ -342,6 +338,9 @@ __device__ void decode_tail(const DecodeArgs& p, uint8_t* smem, int b, int h, in
     }
     rec[4 + d] = a;
   }
+  // the staged rows are dead: order these generic-proxy accesses before any
+  // later tile copy (async proxy) into the same shared memory
+  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
   if (p.append) {
     const int r = L & 127;
     __half* kw = p.tail_w + (((int64_t)b * 2 + 0) * p.Hkv + h) * (int64_t)(kTile * kHeadDim) + (int64_t)r * kHeadDim;
@@ -387,155 +386,50 @@ __device__ __forceinline__ bool issue_unit(const DecodeArgs& p, uint8_t* stage_b
   return ok;
 }
 
-// One segment: full tiles [t_begin, t_end) of sequence b (length L), KV head
-// h, by the whole CTA; writes one partial record per query head at
-// recs + g * 132.  With several queries per sequence the last full tile can
-// hold query positions: there each (query, head) column masks the tokens
-// after its own query.
-// Work units (tile, part) go round-robin over the warps starting at warp
-// `woff`, so a CTA that runs several segments keeps its warps level.  `rearm`:
-// the barriers were used by an earlier segment and are invalidated first.
-// Returns false if a copy timed out (the status is set).
+// The tile loop of one warp: work units u0, u0 + ustep, ... (n_mine of them;
+// unit = (tile, part), tiles counted from t_begin) of sequence b, KV head h,
+// streamed through this warp's private 2-stage ring and folded into the warp's
+// online-softmax state (acc in the rotated domain, running max and sum per
+// query-head column).  kbase: how many units this warp's ring has carried since
+// its barriers were initialised (unit k uses stage (kbase + k) % 2 and waits for
+// phase parity ((kbase + k) / 2) % 2).  Returns the unit whose copy timed out,
+// or -1.
 template <int KB, int VB>
-__device__ __forceinline__ bool decode_segment(const DecodeArgs& p, uint8_t* smem, int b, int h, int grp, int L,
-                                               int t_begin, int t_end, int woff, bool rearm, float* recs) {
+__device__ __forceinline__ int run_units(const DecodeArgs& p, uint8_t* stage_base, uint64_t* my_bars, float* scr,
+                                         float* tokbuf, int b, int h, int t_begin, int kbase, int u0, int ustep,
+                                         int n_mine,
+                                         const float (&qr)[32], float coef0, float coef1, int mask_tile,
+                                         const int (&climit)[2], float (&acc)[8][4], float (&mrun)[2],
+                                         float (&lsum)[2]) {
   using T = DecodeTraits<KB, VB>;
   constexpr int U = T::U, MT = T::MT;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + T::kBarOff);
-  float* qrot = reinterpret_cast<float*>(smem + T::kQrotOff);
-  float* invsig = reinterpret_cast<float*>(smem + T::kInvSigOff);
-
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  if (t_begin >= t_end) return true;
-
-  if (tid == 0) {
-    for (int i = 0; i < kDWarps * kDStages; ++i) {
-      if (rearm) mbar_inval(&bars[i]);
-      mbar_init(&bars[i], 1);
-    }
-    fence_barrier_init();
-  }
-
-  // ---- q H for the group's (query, head) columns, scaled by a power of two so |q H| <= 1 (a6)
-  {
-    const int g = tid >> 4, part = tid & 15;
-    float x[8];
-    int64_t qrow;
-    int qi;
-    if (col_row(p, b, h, grp, g, &qrow, &qi)) {
-      const uint4 raw = __ldg(reinterpret_cast<const uint4*>(p.q + qrow + part * 8));
-      const __half2* hp = reinterpret_cast<const __half2*>(&raw);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float2 f = __half22float2(hp[i]);
-        x[2 * i] = f.x;
-        x[2 * i + 1] = f.y;
-      }
-    } else {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) x[i] = 0.f;
-    }
-#pragma unroll
-    for (int hl = 1; hl < 8; hl <<= 1)
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-        if ((i & hl) == 0) {
-          const float a = x[i], c = x[i + hl];
-          x[i] = a + c;
-          x[i + hl] = a - c;
-        }
-#pragma unroll
-    for (int m = 1; m < 16; m <<= 1) {
-      const bool up = (lane & m) != 0;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float y = __shfl_xor_sync(0xffffffffu, x[i], m);
-        x[i] = up ? (y - x[i]) : (x[i] + y);
-      }
-    }
-    float mx = 0.f;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) mx = fmaxf(mx, fabsf(x[i]));
-#pragma unroll
-    for (int m = 1; m < 16; m <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, m));
-    int e = 0;
-    if (mx > 0.f) frexpf(mx, &e);
-    const float sig = ldexpf(1.f, -e);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) qrot[g * 128 + part * 8 + i] = x[i] * sig;
-    if (part == 0) invsig[g] = ldexpf(1.f, e);
-  }
-  __syncthreads();
-
-  // ---- per-warp state
-  const int g8 = lane >> 2, c = lane & 3;
-#if !KVARN_D_QR_SMEM
-  float qr[32];   // q H of head g8 at channels 16kt + 2c + {0,1,8,9}
-#pragma unroll
-  for (int kt = 0; kt < 8; ++kt) {
-    const float2 lo = *reinterpret_cast<const float2*>(&qrot[g8 * 128 + 16 * kt + 2 * c]);
-    const float2 hi = *reinterpret_cast<const float2*>(&qrot[g8 * 128 + 16 * kt + 2 * c + 8]);
-    qr[4 * kt] = lo.x;
-    qr[4 * kt + 1] = lo.y;
-    qr[4 * kt + 2] = hi.x;
-    qr[4 * kt + 3] = hi.y;
-  }
-#endif
-  // causal limits (last token index attended inside the last full tile) of
-  // this lane's columns 2c, 2c + 1: query i sits at position L - qlen + i
-  const int mask_tile = p.qlen > 1 ? (L >> 7) - 1 : -1;
-  int climit[2] = {kTile - 1, kTile - 1};
-  if (mask_tile >= 0) {
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      int64_t row;
-      int qi;
-      if (col_row(p, b, h, grp, 2 * c + j, &row, &qi)) climit[j] = L - p.qlen + qi - kTile * mask_tile;
-    }
-  }
-#if !KVARN_D_QR_SMEM
-  __syncthreads();   // every warp holds its q H: the q H buffer now serves as per-warp token-scale scratch
-  float* tokbuf = qrot + warp * 256;   // [2 (K, V)][8 (g8)][16 (mt, ri)]
-#else
-  float* tokbuf = reinterpret_cast<float*>(smem + T::kTokOff) + warp * 256;
-#endif
-  const float coef0 = p.sm_scale * kLog2e * (1.f / 128.f) * invsig[2 * c];
-  const float coef1 = p.sm_scale * kLog2e * (1.f / 128.f) * invsig[2 * c + 1];
-  float* scr = reinterpret_cast<float*>(smem + T::kScrOff) + warp * kHeadDim;
-
-  float acc[8][4];
-#pragma unroll
-  for (int i = 0; i < 8; ++i)
-#pragma unroll
-    for (int r = 0; r < 4; ++r) acc[i][r] = 0.f;
-  float mrun[2] = {-INFINITY, -INFINITY}, lsum[2] = {0.f, 0.f};
-
-  // work units of this segment: (tile, part), part in [0, U); warp takes every 4th from u0
-  const int n_units = (t_end - t_begin) * U;
-  const int u0 = (warp - woff + kDWarps) % kDWarps;
-  const int n_mine = u0 < n_units ? (n_units - u0 + kDWarps - 1) / kDWarps : 0;
-  uint8_t* stage_base = smem + warp * kDStages * T::kStage;
-  uint64_t* my_bars = bars + warp * kDStages;
+  const int lane = threadIdx.x & 31, g8 = lane >> 2, c = lane & 3;
   const int32_t* btab = p.block_table + (int64_t)b * p.max_blocks;
-
-  bool ok0 = n_mine > 0 ? issue_unit<KB, VB>(p, stage_base, my_bars, 0, u0, btab[t_begin + u0 / U], h, lane)
-                        : false;
-  bool ok1 = n_mine > 1 ? issue_unit<KB, VB>(p, stage_base, my_bars, 1, u0 + kDWarps,
-                                             btab[t_begin + (u0 + kDWarps) / U], h, lane)
-                        : false;
+  // ok0 / ok1: the unit now in flight in stage 0 / 1 has a valid block
+  bool ok0 = false, ok1 = false;
+  if (n_mine > 0) {
+    const bool o = issue_unit<KB, VB>(p, stage_base, my_bars, kbase, u0, btab[t_begin + u0 / U], h, lane);
+    if (kbase & 1) ok1 = o; else ok0 = o;
+  }
+  if (n_mine > 1) {
+    const bool o = issue_unit<KB, VB>(p, stage_base, my_bars, kbase + 1, u0 + ustep,
+                                      btab[t_begin + (u0 + ustep) / U], h, lane);
+    if (kbase & 1) ok0 = o; else ok1 = o;
+  }
   int k_fail = -1;
 
   for (int k = 0; k < n_mine; ++k) {
-    const int stg = k & 1;
+    const int kg = kbase + k;
+    const int stg = kg & 1;
     // block id of unit k + 2, loaded now so it is in hand when that copy is issued
-    const int32_t blk_next = k + 2 < n_mine ? btab[t_begin + (u0 + (k + 2) * kDWarps) / U] : 0;
-    if (!__all_sync(0xffffffffu, mbar_wait_bounded(&my_bars[stg], (k >> 1) & 1))) {
+    const int32_t blk_next = k + 2 < n_mine ? btab[t_begin + (u0 + (k + 2) * ustep) / U] : 0;
+    if (!__all_sync(0xffffffffu, mbar_wait_bounded(&my_bars[stg], (kg >> 1) & 1))) {
       if (lane == 0) report_status(p.status, KVARN_DEV_TIMEOUT);
       k_fail = k;
       break;
     }
     const bool tile_ok = stg == 0 ? ok0 : ok1;
-    const int part = (u0 + k * kDWarps) % U;
+    const int part = (u0 + k * ustep) % U;
     const uint8_t* st = stage_base + stg * T::kStage;
     if (tile_ok) {
       const uint8_t* rk = st + T::kUnitK + T::kUnitV;   // K scale record, V record follows
@@ -597,15 +491,8 @@ __device__ __forceinline__ bool decode_segment(const DecodeArgs& p, uint8_t* sme
       for (int kt = 0; kt < 8; ++kt) {
         const float2 s01 = *reinterpret_cast<const float2*>(&scr[16 * kt + 2 * c]);
         const float2 s89 = *reinterpret_cast<const float2*>(&scr[16 * kt + 2 * c + 8]);
-#if KVARN_D_QR_SMEM
-        const float2 qlo = *reinterpret_cast<const float2*>(&qrot[g8 * 128 + 16 * kt + 2 * c]);
-        const float2 qhi = *reinterpret_cast<const float2*>(&qrot[g8 * 128 + 16 * kt + 2 * c + 8]);
-        const float x0 = qlo.x * s01.x, x1 = qlo.y * s01.y;
-        const float x8 = qhi.x * s89.x, x9 = qhi.y * s89.y;
-#else
         const float x0 = qr[4 * kt] * s01.x, x1 = qr[4 * kt + 1] * s01.y;
         const float x8 = qr[4 * kt + 2] * s89.x, x9 = qr[4 * kt + 3] * s89.y;
-#endif
         const __half2 h01 = __floats2half2_rn(x0, x1);
         const __half2 h89 = __floats2half2_rn(x8, x9);
         const float2 f01 = __half22float2(h01), f89 = __half22float2(h89);
@@ -688,7 +575,7 @@ __device__ __forceinline__ bool decode_segment(const DecodeArgs& p, uint8_t* sme
         mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
         mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
       }
-      if (t_begin + (u0 + k * kDWarps) / U == mask_tile) {   // warp-uniform: the tile holding query positions
+      if (t_begin + (u0 + k * ustep) / U == mask_tile) {   // warp-uniform: the tile holding query positions
         mx0 = -INFINITY;
         mx1 = -INFINITY;
 #pragma unroll
@@ -789,18 +676,151 @@ __device__ __forceinline__ bool decode_segment(const DecodeArgs& p, uint8_t* sme
           acc[mt][2 * ri + 1] = fmaf(acc[mt][2 * ri + 1], al1, vcs * fmaf(svr, O[mt][2 * ri + 1], zp1));
         }
     }
+    // the stage's generic reads are ordered before the async-proxy refill
+    asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
     __syncwarp();
     if (k + 2 < n_mine) {
-      const bool okn = issue_unit<KB, VB>(p, stage_base, my_bars, k + 2, u0 + (k + 2) * kDWarps, blk_next, h, lane);
+      const bool okn = issue_unit<KB, VB>(p, stage_base, my_bars, kg + 2, u0 + (k + 2) * ustep, blk_next, h, lane);
       if (stg == 0) ok0 = okn; else ok1 = okn;
     }
   }
 
   if (k_fail >= 0) {
-    // let the copies still in flight land before this CTA's shared memory is released
-    (void)mbar_wait_bounded(&my_bars[k_fail & 1], (k_fail >> 1) & 1);
-    if (k_fail + 1 < n_mine) (void)mbar_wait_bounded(&my_bars[(k_fail + 1) & 1], ((k_fail + 1) >> 1) & 1);
+    // let the copies still in flight land before the shared memory is released
+    const int kf = kbase + k_fail;
+    (void)mbar_wait_bounded(&my_bars[kf & 1], (kf >> 1) & 1);
+    if (k_fail + 1 < n_mine) (void)mbar_wait_bounded(&my_bars[(kf + 1) & 1], ((kf + 1) >> 1) & 1);
   }
+
+  return k_fail;
+}
+
+// One segment: full tiles [t_begin, t_end) of sequence b (length L), KV head
+// h, by the whole CTA; writes one partial record per query head at
+// recs + g * 132.  With several queries per sequence the last full tile can
+// hold query positions: there each (query, head) column masks the tokens
+// after its own query.
+// Work units (tile, part) go round-robin over the warps starting at warp
+// `woff`, so a CTA that runs several segments keeps its warps level.  `rearm`:
+// the barriers were used by an earlier segment and are invalidated first.
+// Returns false if a copy timed out (the status is set).
+template <int KB, int VB>
+__device__ __forceinline__ bool decode_segment(const DecodeArgs& p, uint8_t* smem, int b, int h, int grp, int L,
+                                               int t_begin, int t_end, int woff, bool rearm, float* recs) {
+  using T = DecodeTraits<KB, VB>;
+  constexpr int U = T::U;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + T::kBarOff);
+  float* qrot = reinterpret_cast<float*>(smem + T::kQrotOff);
+  float* invsig = reinterpret_cast<float*>(smem + T::kInvSigOff);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (t_begin >= t_end) return true;
+
+  if (tid == 0) {
+    for (int i = 0; i < kDWarps * kDStages; ++i) {
+      if (rearm) mbar_inval(&bars[i]);
+      mbar_init(&bars[i], 1);
+    }
+    fence_barrier_init();
+  }
+
+  // ---- q H for the group's (query, head) columns, scaled by a power of two so |q H| <= 1 (a6)
+  {
+    const int g = tid >> 4, part = tid & 15;
+    float x[8];
+    int64_t qrow;
+    int qi;
+    if (col_row(p, b, h, grp, g, &qrow, &qi)) {
+      const uint4 raw = __ldg(reinterpret_cast<const uint4*>(p.q + qrow + part * 8));
+      const __half2* hp = reinterpret_cast<const __half2*>(&raw);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 f = __half22float2(hp[i]);
+        x[2 * i] = f.x;
+        x[2 * i + 1] = f.y;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) x[i] = 0.f;
+    }
+#pragma unroll
+    for (int hl = 1; hl < 8; hl <<= 1)
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        if ((i & hl) == 0) {
+          const float a = x[i], c = x[i + hl];
+          x[i] = a + c;
+          x[i + hl] = a - c;
+        }
+#pragma unroll
+    for (int m = 1; m < 16; m <<= 1) {
+      const bool up = (lane & m) != 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float y = __shfl_xor_sync(0xffffffffu, x[i], m);
+        x[i] = up ? (y - x[i]) : (x[i] + y);
+      }
+    }
+    float mx = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) mx = fmaxf(mx, fabsf(x[i]));
+#pragma unroll
+    for (int m = 1; m < 16; m <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, m));
+    int e = 0;
+    if (mx > 0.f) frexpf(mx, &e);
+    const float sig = ldexpf(1.f, -e);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) qrot[g * 128 + part * 8 + i] = x[i] * sig;
+    if (part == 0) invsig[g] = ldexpf(1.f, e);
+  }
+  __syncthreads();
+
+  // ---- per-warp state
+  const int g8 = lane >> 2, c = lane & 3;
+  float qr[32];   // q H of head g8 at channels 16kt + 2c + {0,1,8,9}
+#pragma unroll
+  for (int kt = 0; kt < 8; ++kt) {
+    const float2 lo = *reinterpret_cast<const float2*>(&qrot[g8 * 128 + 16 * kt + 2 * c]);
+    const float2 hi = *reinterpret_cast<const float2*>(&qrot[g8 * 128 + 16 * kt + 2 * c + 8]);
+    qr[4 * kt] = lo.x;
+    qr[4 * kt + 1] = lo.y;
+    qr[4 * kt + 2] = hi.x;
+    qr[4 * kt + 3] = hi.y;
+  }
+  // causal limits (last token index attended inside the last full tile) of
+  // this lane's columns 2c, 2c + 1: query i sits at position L - qlen + i
+  const int mask_tile = p.qlen > 1 ? (L >> 7) - 1 : -1;
+  int climit[2] = {kTile - 1, kTile - 1};
+  if (mask_tile >= 0) {
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      int64_t row;
+      int qi;
+      if (col_row(p, b, h, grp, 2 * c + j, &row, &qi)) climit[j] = L - p.qlen + qi - kTile * mask_tile;
+    }
+  }
+  __syncthreads();   // every warp holds its q H: the q H buffer now serves as per-warp token-scale scratch
+  float* tokbuf = qrot + warp * 256;   // [2 (K, V)][8 (g8)][16 (mt, ri)]
+  const float coef0 = p.sm_scale * kLog2e * (1.f / 128.f) * invsig[2 * c];
+  const float coef1 = p.sm_scale * kLog2e * (1.f / 128.f) * invsig[2 * c + 1];
+  float* scr = reinterpret_cast<float*>(smem + T::kScrOff) + warp * kHeadDim;
+
+  float acc[8][4];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int r = 0; r < 4; ++r) acc[i][r] = 0.f;
+  float mrun[2] = {-INFINITY, -INFINITY}, lsum[2] = {0.f, 0.f};
+
+  // work units of this segment: (tile, part), part in [0, U); warp takes every 4th from u0
+  const int n_units = (t_end - t_begin) * U;
+  const int u0 = (warp - woff + kDWarps) % kDWarps;
+  const int n_mine = u0 < n_units ? (n_units - u0 + kDWarps - 1) / kDWarps : 0;
+  uint8_t* stage_base = smem + warp * kDStages * T::kStage;
+  uint64_t* my_bars = bars + warp * kDStages;
+
+  const int k_fail = run_units<KB, VB>(p, stage_base, my_bars, scr, tokbuf, b, h, t_begin, 0, u0, kDWarps, n_mine, qr,
+                                       coef0, coef1, mask_tile, climit, acc, mrun, lsum);
 
   // ---- merge the four warps and write the partial (m, l, acc) per head
 #pragma unroll
@@ -941,9 +961,9 @@ __device__ void sk_locate(const DecodeArgs& p, int cta, int P, long long* W_out,
 // tail record from its own slot.  One warp per head; lane owns channels
 // 4*lane .. 4*lane + 3.  Records written by other CTAs are read with
 // ld.global.cg (L2), never through L1.
-__device__ void combine_pair(const DecodeArgs& p, int b, int h, int grp, int L, bool valid, long long pst, int nt,
-                             long long W, int P) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+__device__ void combine_columns(const DecodeArgs& p, int b, int h, int grp, int L, bool valid, long long pst, int nt,
+                                long long W, int P, int col0, int col1) {
+  const int lane = threadIdx.x & 31;
   const int pair = (b * p.Hkv + h) * p.ngrp + grp;   // work pair: (sequence, KV head, column group)
   // CTAs whose ranges meet the tiles: owner(pst) .. owner(pst + nt - 1).  With
   // W >= P every CTA range is non-empty, so each of them wrote a record.
@@ -959,7 +979,7 @@ __device__ void combine_pair(const DecodeArgs& p, int b, int h, int grp, int L, 
 #pragma unroll
   for (int k = 0; k < 2; ++k) {
     int qi;
-    gh[k] = warp + kDWarps * k;
+    gh[k] = k == 0 ? col0 : col1;
     hl[k] = col_row(p, b, h, grp, gh[k], &orow[k], &qi);
   }
   if (!hl[0]) return;
@@ -1052,6 +1072,13 @@ __device__ void combine_pair(const DecodeArgs& p, int b, int h, int grp, int L, 
     __half* o = p.out + orow[k] + 4 * lane;
     *reinterpret_cast<uint2*>(o) = make_uint2(h2_as_u32(o01), h2_as_u32(o23));
   }
+}
+
+// The CTA version: warp w merges columns w and w + 4.
+__device__ __forceinline__ void combine_pair(const DecodeArgs& p, int b, int h, int grp, int L, bool valid,
+                                             long long pst, int nt, long long W, int P) {
+  const int warp = threadIdx.x >> 5;
+  combine_columns(p, b, h, grp, L, valid, pst, nt, W, P, warp, warp + kDWarps);
 }
 
 // ------------------------------------------------------------------ main kernel
@@ -1163,6 +1190,7 @@ __global__ void __launch_bounds__(kDThreads, KVARN_D_MIN_CTAS) decode_kernel(con
     }
   }
 }
+
 
 template <int KB, int VB>
 cudaError_t launch_d(const DecodeArgs& p, cudaStream_t stream) {

@@ -35,7 +35,7 @@ struct DecodeArgs {
   const int32_t* block_table;
   const int32_t* seq_lens;
   __half* out;
-  float* ws;            // tile partial records [(B * Hkv + kDecodeMaxCtas) * G]
+  float* ws;            // tile partial records [(B * Hkv * ngrp + kDecodeMaxCtas) * C]
   float* ws_tail;       // tail partial records [B * Hkv * G]
   int* counters;        // B * Hkv arrival counters (zeroed by each call)
   int B, Hq, Hkv, G, max_blocks;

@@ -34,14 +34,15 @@ def libs():
 
 def test_decode_wait_timeout_is_reported_and_device_stays_usable(libs):
     K, stall = libs
-    # more work units than decode CTAs, so that CTA 0 (whose first copy stalls) has a range
-    w = inputs.make_decode_workload("timeout", [150 * 128 + 9, 60 * 128, 300], 16, 2, seed=990, pool_blocks=220)
+    # more work units than decode warps (4 per CTA, 2 CTAs per SM), so that warp 0
+    # of CTA 0 (whose first copy stalls) has a range
+    w = inputs.make_decode_workload("timeout", [200 * 128 + 9, 180 * 128, 300], 16, 4, seed=990, pool_blocks=390)
     cfg = K.config()
     dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
-    packed, scales = K.alloc_cache(cfg, w.num_blocks, 2)
+    packed, scales = K.alloc_cache(cfg, w.num_blocks, 4)
     K.quantize_tiles(dev(w.k_full), dev(w.v_full), dev(w.slot_mapping), packed, scales, cfg)
     q, tail, bt, sl = dev(w.q), dev(w.tail), dev(w.block_table), dev(w.seq_lens)
-    d = K.dims(w.num_seqs, 16, 2, w.max_blocks_per_seq, w.num_blocks)
+    d = K.dims(w.num_seqs, 16, 4, w.max_blocks_per_seq, w.num_blocks)
     ws = torch.zeros(K.decode_workspace_bytes(cfg, d), dtype=torch.uint8, device="cuda")
     out = torch.empty_like(q)
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
@@ -57,6 +58,6 @@ def test_decode_wait_timeout_is_reported_and_device_stays_usable(libs):
     got = K.decode_attention(q, packed, scales, tail, bt, sl, cfg, workspace=ws, dev_status=status)
     torch.cuda.synchronize()
     assert int(status.item()) == 0
-    ref = O.decode(w.q, packed.cpu().numpy(), scales.cpu().numpy(), w.tail, w.block_table, w.seq_lens, 2, 4, 2)
+    ref = O.decode(w.q, packed.cpu().numpy(), scales.cpu().numpy(), w.tail, w.block_table, w.seq_lens, 4, 4, 2)
     err = np.abs(got.cpu().numpy().astype(np.float64) - ref.astype(np.float64))
     assert np.all(err <= np.maximum(2e-3, np.spacing(np.abs(ref)).astype(np.float64)))
