@@ -95,6 +95,14 @@ class ClockSampler:
             self._t.start()
         return self
 
+    def start_region(self, timeout_s: float = 1.0):
+        """Wait until the sampler runs, then keep only samples taken from now on."""
+        t0 = time.perf_counter()
+        while self._ok and not self.samples and time.perf_counter() - t0 < timeout_s:
+            time.sleep(0.0002)
+        self.samples.clear()
+        self.reasons.clear()
+
     def __exit__(self, *a):
         if self._ok:
             self._stop.set()
@@ -227,10 +235,13 @@ def run_gpu(args):
         dist.barrier()
     torch.cuda.synchronize()
     with sampler:
+        sampler.start_region()
         e0.record(stream)
         for _ in range(args.steps):
             step()
         e1.record(stream)
+        while not e1.query():          # yield to the sampler thread while the GPU runs
+            time.sleep(0.0002)
         torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
