@@ -507,7 +507,19 @@ __device__ __forceinline__ int run_units(const DecodeArgs& p, uint8_t* stage_bas
         ql0[kt] = h2_as_u32(l01);
         ql1[kt] = h2_as_u32(l89);
       }
-      __syncwarp();   // scr is rewritten by the next unit
+      __syncwarp();   // the K channel scales in scr are dead
+      // V channel scales 2^Lc_v once per channel (4 per lane) into scr, read
+      // back in the accumulator layout (channel 16mt + g8 + 8ri at g8 * 16 + 2mt + ri)
+      {
+        const float2 v01 = __half22float2(*reinterpret_cast<const __half2*>(lcv + 4 * lane));
+        const float2 v23 = __half22float2(*reinterpret_cast<const __half2*>(lcv + 4 * lane + 2));
+        const float vv[4] = {v01.x, v01.y, v23.x, v23.y};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int d = 4 * lane + i;
+          scr[(d & 7) * 16 + (d >> 4) * 2 + ((d >> 3) & 1)] = ex2_fast(vv[i]);
+        }
+      }
       qsum += __shfl_xor_sync(0xffffffffu, qsum, 1);
       qsum += __shfl_xor_sync(0xffffffffu, qsum, 2);
       const float qs0 = __shfl_sync(0xffffffffu, qsum, (2 * c) * 4);
@@ -666,11 +678,18 @@ __device__ __forceinline__ int run_units(const DecodeArgs& p, uint8_t* stage_bas
       const float zp0 = zv * tvf * ps0, zp1 = zv * tvf * ps1;
       const float sv0 = sv * tvf * (16777216.f / static_cast<float>(1 << CodeShift<VB>::kBase));
       const float sv1 = sv0 * (1.f / static_cast<float>(1 << CodeShift<VB>::kSRow));
+      __syncwarp();   // the V channel scales are in scr
+      float vcsv[16];
+#pragma unroll
+      for (int k4 = 0; k4 < 4; ++k4) {
+        const float4 x = *reinterpret_cast<const float4*>(&scr[g8 * 16 + 4 * k4]);
+        vcsv[4 * k4] = x.x; vcsv[4 * k4 + 1] = x.y; vcsv[4 * k4 + 2] = x.z; vcsv[4 * k4 + 3] = x.w;
+      }
 #pragma unroll
       for (int mt = 0; mt < 8; ++mt)
 #pragma unroll
         for (int ri = 0; ri < 2; ++ri) {
-          const float vcs = ex2_fast(hf(lcv, 16 * mt + g8 + 8 * ri));
+          const float vcs = vcsv[2 * mt + ri];
           const float svr = ri ? sv1 : sv0;   // step with the codes' placement undone, per row half
           acc[mt][2 * ri] = fmaf(acc[mt][2 * ri], al0, vcs * fmaf(svr, O[mt][2 * ri], zp0));
           acc[mt][2 * ri + 1] = fmaf(acc[mt][2 * ri + 1], al1, vcs * fmaf(svr, O[mt][2 * ri + 1], zp1));
@@ -879,13 +898,13 @@ __device__ __forceinline__ bool decode_segment(const DecodeArgs& p, uint8_t* sme
 // kTailUnits for the fp16 tail (which also carries an empty or invalid
 // sequence, so every pair is owned).  The tail, and usually the merge of the
 // pair, fall to the CTA owning the pair's last unit; weighting them as
-// several tiles keeps that CTA's range shorter.  A pair with no tail rows
+// several tiles keeps that CTA's range shorter (14 measured best of 4-18).  A pair with no tail rows
 // (seq_len a multiple of 128, nothing appended) weighs kTailUnitsEmpty: the
 // merge and a segment restart only.
 // A tail that an appended token fills is also quantised, K and V as two more
 // work items of kFillUnits each after the tail (rotation recomputed), so that
 // up to three CTAs share a fill.  Each item falls to the CTA holding its last unit.
-constexpr int kTailUnits = 9;
+constexpr int kTailUnits = 14;
 constexpr int kTailUnitsEmpty = 3;
 constexpr int kFillUnits = 16;
 
