@@ -8,17 +8,20 @@
 //             a +-1 fp16 H16) and the 8-group factor is an in-register
 //             butterfly across the eight mma results each lane holds;
 //   3 normalise  N passes of channel RMS then token RMS in base-2 log space:
-//             A = R*R stays in registers; each pass is packed f32x2 FMAs, a
-//             warp reduce-scatter and (for channels) a 4-warp shared sum;
+//             A = R*R stays in registers; each pass is packed f32x2 FMAs and
+//             a sum of the per-thread partials through shared memory
+//             (channels: over the 16 threads of the CTA that hold a channel;
+//             tokens: over the 8 lanes of a warp that hold a token);
 //   4 quantise   Z = (R * fp32(2^-Lt)) * fp32(2^-Lc) from the stored fp16
 //             log-scales, one zero/step per tile from min/max, codes =
 //             clamp(rne((Z - zero) / step)), the quotient formed in fp32 as
 //             Z * (1/step) - zero * (1/step) (one FMA per element);
 //   5 pack    codes in the decode's mma fragment order, 16-byte stores.
-// The K-side rotation uses X as the mma A operand and the V side as the B
-// operand, so after stage 2 each lane holds exactly the elements of the
-// decode kernel's mma fragments (K: rows tokens; V: rows channels): codes are
-// packed in registers and written with no cross-lane traffic.
+// The rotation uses H16 as the mma A operand and X as the B operand, so after
+// stage 2 each lane holds exactly the elements of the decode kernel's V-side
+// mma fragments (rows channels): V codes are packed in registers with no
+// cross-lane traffic, and K codes (rows tokens) after one movmatrix transpose
+// per 8x8 block of code pairs.
 // Used by the quantise-on-write kernel and by the decode kernel's append path.
 #pragma once
 #include "common.cuh"
@@ -30,16 +33,40 @@ namespace qt {
 constexpr int kQThreads = 128;
 constexpr int kBox = 128 * 128;       // one 64-channel box: 128 rows of 128 bytes
 
-// Per-CTA scratch of one tile's normalisation and quantisation.
+// Row stride (floats) of the channel-pass exchange: 128 + 4, so that the 8
+// lanes of a quarter-warp writing 16 bytes each (4 rows x 2 column blocks) hit
+// distinct banks.
+constexpr int kXchStride = kHeadDim + 4;
+
+// Row stride (floats) of a warp's token-pass exchange (8 rows of 32 partials):
+// 32 + 4, so the 16-byte stores of a quarter-warp (2 rows x 4 column blocks)
+// and the column reads hit distinct banks.  8 such rows fit in the warp's own
+// 4 channel-exchange rows.
+constexpr int kTokStride = 32 + 4;
+static_assert(8 * kTokStride <= 4 * kXchStride, "token exchange inside the warp's channel rows");
+
+// Per-CTA scratch of one tile's normalisation and quantisation.  Channels are
+// kept in the permuted order j = g*16 + 2a + ri of channel 16a + g + 8ri (the
+// order in which a lane of the register layout holds its 16 channels).
 struct QuantScratch {
-  float red[4][kHeadDim];                // per-warp channel partial sums
-  alignas(16) float u[kHeadDim];         // channel weights 2^(-2 lc), channel 16a + g + 8ri at g*16 + 2a + ri
+  union {
+    // normalisation: channel partial sums, row (warp, c) x permuted channel;
+    // during the token pass, rows 4w .. 4w+3 hold warp w's token partials
+    alignas(16) float xch[16 * kXchStride];
+    // quantisation (after the last pass)
+    struct {
+      float mt[kTile];                     // fp32(2^-Lt)
+      float mc[kHeadDim];                  // fp32(2^-Lc)
+      float zmin[4], zmax[4];
+      alignas(16) uint8_t rec[kScaleRec];  // staged scale record
+    } q;
+  };
+  alignas(16) float u[kHeadDim];         // channel weights 2^(-2 lc), permuted order
   alignas(16) float wb[4][32];           // per-warp token-weight exchange
-  float mt[kTile];                       // fp32(2^-Lt)
-  float mc[kHeadDim];                    // fp32(2^-Lc)
-  float zmin[4], zmax[4];
-  alignas(16) uint8_t rec[kScaleRec];    // staged scale record
 };
+
+// channel of permuted index j = g*16 + 2a + ri
+__device__ __forceinline__ int perm_channel(int j) { return 16 * ((j >> 1) & 7) + (j >> 4) + 8 * (j & 1); }
 
 // Tensor memory can hold a tile's rotated R (fp32, 128 lanes x 128 columns =
 // 64 KB) from the rotation until quantisation, so R is computed once.
@@ -91,30 +118,6 @@ __device__ __forceinline__ void fwht8x2(float2 (&v)[8]) {
         v[i + hl] = __fadd2_rn(a, make_float2(-b.x, -b.y));
       }
     }
-  }
-}
-
-// One reduce-scatter step across lanes (lane ^ mask): the first N/2 entries
-// of v end up holding the half this lane keeps, summed with its partner's.
-template <int N>
-__device__ __forceinline__ void rs_step(float* v, int mask, int lane) {
-  const bool up = (lane & mask) != 0;
-  float keep[N / 2], recv[N / 2];
-#pragma unroll
-  for (int i = 0; i < N / 2; ++i) {
-    const float send = up ? v[i] : v[i + N / 2];
-    keep[i] = up ? v[i + N / 2] : v[i];
-    recv[i] = __shfl_xor_sync(0xffffffffu, send, mask);
-  }
-  if constexpr (N / 2 >= 2) {   // the adds in f32x2 pairs
-#pragma unroll
-    for (int i = 0; i < N / 2; i += 2) {
-      const float2 r = __fadd2_rn(make_float2(keep[i], keep[i + 1]), make_float2(recv[i], recv[i + 1]));
-      v[i] = r.x;
-      v[i + 1] = r.y;
-    }
-  } else {
-    v[0] = keep[0] + recv[0];
   }
 }
 
@@ -182,51 +185,6 @@ __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.
 
 // ---------------------------------------------------------------- rotation
 
-// K side: thread holds R at t = 16*(2w+ml) + g + 8*ri, d = 16*a + 8*nb + 2*c + rj
-// in R[((ml*8 + a)*2 + nb)*4 + 2*ri + rj]   (g = lane/4, c = lane%4).
-__device__ __forceinline__ void rotate_k(uint32_t xs, int warp, int lane, float (&R)[128]) {
-  const int g = lane >> 2, c = lane & 3;
-  uint32_t hb0[2], hb1[2];
-#pragma unroll
-  for (int nb = 0; nb < 2; ++nb) {
-    const int n = 8 * nb + g;
-    hb0[nb] = h16_pair(2 * c, n, 2 * c + 1, n);
-    hb1[nb] = h16_pair(2 * c + 8, n, 2 * c + 9, n);
-  }
-  const int mi = lane >> 3;
-#pragma unroll
-  for (int ml = 0; ml < 2; ++ml) {
-    const int row = 16 * (2 * warp + ml) + (lane & 7) + 8 * (mi & 1);
-    float C[8][2][4];
-#pragma unroll
-    for (int a = 0; a < 8; ++a) {
-      uint32_t a0, a1, a2, a3;
-      ldmatrix_x4(xs + xoff(row, 2 * a + (mi >> 1)), a0, a1, a2, a3);
-#pragma unroll
-      for (int nb = 0; nb < 2; ++nb) {
-#pragma unroll
-        for (int r = 0; r < 4; ++r) C[a][nb][r] = 0.f;
-        mma_f16(C[a][nb], a0, a1, a2, a3, hb0[nb], hb1[nb]);
-      }
-    }
-#pragma unroll
-    for (int nb = 0; nb < 2; ++nb) {
-#pragma unroll
-      for (int r = 0; r < 4; r += 2) {
-        float2 v[8];
-#pragma unroll
-        for (int a = 0; a < 8; ++a) v[a] = make_float2(C[a][nb][r], C[a][nb][r + 1]);
-        fwht8x2(v);
-#pragma unroll
-        for (int a = 0; a < 8; ++a) {
-          R[((ml * 8 + a) * 2 + nb) * 4 + r] = v[a].x;
-          R[((ml * 8 + a) * 2 + nb) * 4 + r + 1] = v[a].y;
-        }
-      }
-    }
-  }
-}
-
 // V side: thread holds R at t = 8*(4w+ntl) + 2*c + rj, d = 16*a + g + 8*ri
 // in R[(ntl*8 + a)*4 + 2*ri + rj].
 __device__ __forceinline__ void rotate_v(uint32_t xs, int warp, int lane, float (&R)[128]) {
@@ -269,14 +227,6 @@ __device__ __forceinline__ void rotate_v(uint32_t xs, int warp, int lane, float 
 
 // ---------------------------------------------------------------- the tile
 
-// K tiles use the V tiles' register layout (rows = channels) through the
-// normalisation -- its reductions move about a quarter fewer words between
-// lanes -- and are transposed to the K fragment order when packed.  0 keeps
-// the K-specific layout (rows = tokens) throughout.
-#ifndef KVARN_Q_K_VLAYOUT
-#define KVARN_Q_K_VLAYOUT 1
-#endif
-
 // Where one tile's results go.
 struct TileOut {
   uint8_t* codes;        // this side's code block (2048 * BITS bytes, 16-byte aligned)
@@ -291,13 +241,12 @@ struct TileOut {
 // rotation is run a second time from the staged tile (same arithmetic).
 template <int SIDE, int BITS, bool STASH>
 __device__ __forceinline__ void quantize_tile(const TileOut& o, QuantScratch& sm, uint32_t xs, uint32_t tmem) {
-  constexpr bool KL = SIDE == 0 && KVARN_Q_K_VLAYOUT == 0;   // the K-specific layout
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, c = lane & 3;
 
   // ---- 2. rotate
   float A[128];
-  if (KL) rotate_k(xs, warp, lane, A); else rotate_v(xs, warp, lane, A);
+  rotate_v(xs, warp, lane, A);
   // stash R in this warp's 32 TMEM lanes (lane field: bits 31..16, column: 15..0)
   const uint32_t tr = tmem + (static_cast<uint32_t>(32 * warp) << 16);
   if (STASH) {
@@ -313,39 +262,18 @@ __device__ __forceinline__ void quantize_tile(const TileOut& o, QuantScratch& sm
   }
 
   // ---- 3. normalise
-  constexpr int NT = KL ? 4 : 8;   // tokens per thread
+  constexpr int NT = 8;   // tokens per thread
   float wt[NT];                           // token weights 2^(-2 lt)
 #pragma unroll
   for (int i = 0; i < NT; ++i) wt[i] = 1.f;
   float lt_sum = 1.f, lc_sum = 1.f;   // this thread's token / channel sums of the last pass
 
   for (int it = 0; it < o.iters; ++it) {
-    // channel pass: partial sums over this thread's tokens
-    if (KL) {
-      float s[32];   // index a*4 + nb*2 + rj
-#pragma unroll
-      for (int a = 0; a < 8; ++a)
-#pragma unroll
-        for (int nb = 0; nb < 2; ++nb) {
-          float2 acc = f2(0.f, 0.f);
-#pragma unroll
-          for (int ml = 0; ml < 2; ++ml)
-#pragma unroll
-            for (int ri = 0; ri < 2; ++ri) {
-              const int i = ((ml * 8 + a) * 2 + nb) * 4 + 2 * ri;
-              const float w = wt[ml * 2 + ri];
-              acc = __ffma2_rn(f2(A[i], A[i + 1]), f2(w, w), acc);
-            }
-          s[a * 4 + nb * 2] = acc.x;
-          s[a * 4 + nb * 2 + 1] = acc.y;
-        }
-      rs_step<32>(s, 16, lane);
-      rs_step<16>(s, 8, lane);
-      rs_step<8>(s, 4, lane);
-      *reinterpret_cast<float2*>(&sm.red[warp][16 * g + 2 * c]) = f2(s[0], s[1]);
-      *reinterpret_cast<float2*>(&sm.red[warp][16 * g + 8 + 2 * c]) = f2(s[2], s[3]);
-    } else {
-      float s[16];   // index a*2 + ri
+    // channel pass: partial sums over this thread's 8 tokens for its 16
+    // channels, to row (warp, c) of the exchange in the permuted order (four
+    // 16-byte stores); thread j then sums permuted channel j over the 16 rows
+    {
+      float s[16];   // index a*2 + ri = permuted position within this lane's 16
 #pragma unroll
       for (int a = 0; a < 8; ++a)
 #pragma unroll
@@ -358,54 +286,28 @@ __device__ __forceinline__ void quantize_tile(const TileOut& o, QuantScratch& sm
           }
           s[a * 2 + ri] = acc.x + acc.y;
         }
-      rs_step<16>(s, 2, lane);
-      rs_step<8>(s, 1, lane);
+      float* row = sm.xch + (warp * 4 + c) * kXchStride + g * 16;
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int a = 2 * c + (k >> 1), ri = k & 1;
-        sm.red[warp][16 * a + g + 8 * ri] = s[k];
-      }
+      for (int k4 = 0; k4 < 4; ++k4)
+        *reinterpret_cast<float4*>(row + 4 * k4) = make_float4(s[4 * k4], s[4 * k4 + 1], s[4 * k4 + 2], s[4 * k4 + 3]);
     }
     __syncthreads();
     {
-      const float tot = (sm.red[0][tid] + sm.red[1][tid]) + (sm.red[2][tid] + sm.red[3][tid]);
-      lc_sum = tot;
-      sm.u[KL ? tid : (tid & 7) * 16 + (tid >> 4) * 2 + ((tid >> 3) & 1)] = weight_of_sum(tot);
+      float2 t[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) t[r] = f2(sm.xch[(2 * r) * kXchStride + tid], sm.xch[(2 * r + 1) * kXchStride + tid]);
+#pragma unroll
+      for (int r = 8; r < 16; r += 2)
+        t[(r >> 1) & 3] = __fadd2_rn(t[(r >> 1) & 3], f2(sm.xch[r * kXchStride + tid], sm.xch[(r + 1) * kXchStride + tid]));
+      const float2 t01 = __fadd2_rn(t[0], t[1]), t23 = __fadd2_rn(t[2], t[3]);
+      const float2 tt = __fadd2_rn(t01, t23);
+      lc_sum = tt.x + tt.y;
+      sm.u[tid] = weight_of_sum(lc_sum);
     }
     __syncthreads();
 
     // token pass
-    if (KL) {
-      float2 uu[16];   // (a, nb) -> channels 16a + 8nb + 2c + {0,1}
-#pragma unroll
-      for (int a = 0; a < 8; ++a)
-#pragma unroll
-        for (int nb = 0; nb < 2; ++nb)
-          uu[a * 2 + nb] = *reinterpret_cast<const float2*>(&sm.u[16 * a + 8 * nb + 2 * c]);
-      float s[4];    // index ml*2 + ri
-#pragma unroll
-      for (int ml = 0; ml < 2; ++ml)
-#pragma unroll
-        for (int ri = 0; ri < 2; ++ri) {
-          float2 acc[4] = {f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f)};   // 4 chains for ILP
-#pragma unroll
-          for (int a = 0; a < 8; ++a)
-#pragma unroll
-            for (int nb = 0; nb < 2; ++nb) {
-              const int i = ((ml * 8 + a) * 2 + nb) * 4 + 2 * ri;
-              acc[(a & 1) * 2 + nb] = __ffma2_rn(f2(A[i], A[i + 1]), uu[a * 2 + nb], acc[(a & 1) * 2 + nb]);
-            }
-          const float2 t01 = __fadd2_rn(acc[0], acc[1]), t23 = __fadd2_rn(acc[2], acc[3]);
-          const float2 t = __fadd2_rn(t01, t23);
-          s[ml * 2 + ri] = t.x + t.y;
-        }
-      rs_step<4>(s, 2, lane);
-      rs_step<2>(s, 1, lane);
-      lt_sum = s[0];
-      const float wown = weight_of_sum(s[0]);
-#pragma unroll
-      for (int k = 0; k < 4; ++k) wt[k] = __shfl_sync(0xffffffffu, wown, (lane & ~3) | k);
-    } else {
+    {
       float uu[16];
 #pragma unroll
       for (int k4 = 0; k4 < 4; ++k4) {
@@ -428,11 +330,21 @@ __device__ __forceinline__ void quantize_tile(const TileOut& o, QuantScratch& sm
         s[ntl * 2] = t.x;
         s[ntl * 2 + 1] = t.y;
       }
-      rs_step<8>(s, 16, lane);
-      rs_step<4>(s, 8, lane);
-      rs_step<2>(s, 4, lane);
-      lt_sum = s[0];
-      sm.wb[warp][c * 8 + g] = weight_of_sum(s[0]);
+      // the 8 lanes g = 0..7 of one c hold partials of the same 8 tokens: row
+      // g, columns c*8 .. c*8+7 of this warp's own exchange rows (free until
+      // its next channel pass); lane (g, c) then sums column c*8 + g, i.e.
+      // token (ntl, rj) = (g >> 1, g & 1) of its c
+      float* tx = sm.xch + warp * 4 * kXchStride;
+      *reinterpret_cast<float4*>(tx + g * kTokStride + c * 8) = make_float4(s[0], s[1], s[2], s[3]);
+      *reinterpret_cast<float4*>(tx + g * kTokStride + c * 8 + 4) = make_float4(s[4], s[5], s[6], s[7]);
+      __syncwarp();
+      const float* col = tx + c * 8 + g;
+      float2 t0 = f2(col[0], col[kTokStride]), t1 = f2(col[2 * kTokStride], col[3 * kTokStride]);
+      t0 = __fadd2_rn(t0, f2(col[4 * kTokStride], col[5 * kTokStride]));
+      t1 = __fadd2_rn(t1, f2(col[6 * kTokStride], col[7 * kTokStride]));
+      const float2 tt = __fadd2_rn(t0, t1);
+      lt_sum = tt.x + tt.y;
+      sm.wb[warp][c * 8 + g] = weight_of_sum(lt_sum);
       __syncwarp();
       const float4 w0 = *reinterpret_cast<const float4*>(&sm.wb[warp][c * 8]);
       const float4 w1 = *reinterpret_cast<const float4*>(&sm.wb[warp][c * 8 + 4]);
@@ -442,19 +354,22 @@ __device__ __forceinline__ void quantize_tile(const TileOut& o, QuantScratch& sm
     }
   }
 
+  // the last token pass's exchange rows overlap the quantisation scratch
+  __syncthreads();
+
   // ---- stored fp16 log-scales and their fp32 multipliers
-  const int t_own = KL ? 16 * (2 * warp + ((lane >> 1) & 1)) + g + 8 * (lane & 1)
-                                : 8 * (4 * warp + (lane >> 3)) + 2 * c + ((lane >> 2) & 1);
+  const int t_own = 8 * (4 * warp + (lane >> 3)) + 2 * c + ((lane >> 2) & 1);
+  const int c_own = perm_channel(tid);
   const float lt_own = log2_scale(lt_sum), lc_own = log2_scale(lc_sum);
   const __half Lt16 = __float2half_rn(lt_own);
   const __half Lc16 = __float2half_rn(lc_own);
-  sm.mt[t_own] = __double2float_rn(exp2(-static_cast<double>(__half2float(Lt16))));
-  sm.mc[tid] = __double2float_rn(exp2(-static_cast<double>(__half2float(Lc16))));
-  reinterpret_cast<__half*>(sm.rec)[t_own] = Lt16;
-  reinterpret_cast<__half*>(sm.rec + 256)[tid] = Lc16;
+  sm.q.mt[t_own] = __double2float_rn(exp2(-static_cast<double>(__half2float(Lt16))));
+  sm.q.mc[c_own] = __double2float_rn(exp2(-static_cast<double>(__half2float(Lc16))));
+  reinterpret_cast<__half*>(sm.q.rec)[t_own] = Lt16;
+  reinterpret_cast<__half*>(sm.q.rec + 256)[c_own] = Lc16;
   if (o.dbg != nullptr) {
     o.dbg[t_own] = lt_own;
-    o.dbg[128 + tid] = lc_own;
+    o.dbg[128 + c_own] = lc_own;
   }
   __syncthreads();
 
@@ -465,62 +380,36 @@ __device__ __forceinline__ void quantize_tile(const TileOut& o, QuantScratch& sm
     for (int q = 0; q < 4; ++q) tmem_ld32(tr + 32 * q, Z + 32 * q);
     tmem_wait_ld();
   } else {
-    if (KL) rotate_k(xs, warp, lane, Z); else rotate_v(xs, warp, lane, Z);
+    rotate_v(xs, warp, lane, Z);
   }
   float zlo = 3.402823466e38f, zhi = -3.402823466e38f;
-  if (KL) {
-    float mtv[4];
+  float2 mtv[4];
 #pragma unroll
-    for (int ml = 0; ml < 2; ++ml)
+  for (int ntl = 0; ntl < 4; ++ntl) mtv[ntl] = *reinterpret_cast<const float2*>(&sm.q.mt[8 * (4 * warp + ntl) + 2 * c]);
 #pragma unroll
-      for (int ri = 0; ri < 2; ++ri) mtv[ml * 2 + ri] = sm.mt[16 * (2 * warp + ml) + g + 8 * ri];
+  for (int a = 0; a < 8; ++a)
 #pragma unroll
-    for (int a = 0; a < 8; ++a)
+    for (int ri = 0; ri < 2; ++ri) {
+      const float mcv = sm.q.mc[16 * a + g + 8 * ri];
 #pragma unroll
-      for (int nb = 0; nb < 2; ++nb) {
-        const float2 mc2 = *reinterpret_cast<const float2*>(&sm.mc[16 * a + 8 * nb + 2 * c]);
-#pragma unroll
-        for (int ml = 0; ml < 2; ++ml)
-#pragma unroll
-          for (int ri = 0; ri < 2; ++ri) {
-            const int i = ((ml * 8 + a) * 2 + nb) * 4 + 2 * ri;
-            const float m = mtv[ml * 2 + ri];
-            const float2 z = __fmul2_rn(__fmul2_rn(f2(Z[i], Z[i + 1]), f2(m, m)), mc2);
-            Z[i] = z.x;
-            Z[i + 1] = z.y;
-            zlo = min3(zlo, z.x, z.y);
-            zhi = max3(zhi, z.x, z.y);
-          }
+      for (int ntl = 0; ntl < 4; ++ntl) {
+        const int i = (ntl * 8 + a) * 4 + 2 * ri;
+        const float2 z = __fmul2_rn(__fmul2_rn(f2(Z[i], Z[i + 1]), mtv[ntl]), f2(mcv, mcv));
+        Z[i] = z.x;
+        Z[i + 1] = z.y;
+        zlo = min3(zlo, z.x, z.y);
+        zhi = max3(zhi, z.x, z.y);
       }
-  } else {
-    float2 mtv[4];
-#pragma unroll
-    for (int ntl = 0; ntl < 4; ++ntl) mtv[ntl] = *reinterpret_cast<const float2*>(&sm.mt[8 * (4 * warp + ntl) + 2 * c]);
-#pragma unroll
-    for (int a = 0; a < 8; ++a)
-#pragma unroll
-      for (int ri = 0; ri < 2; ++ri) {
-        const float mcv = sm.mc[16 * a + g + 8 * ri];
-#pragma unroll
-        for (int ntl = 0; ntl < 4; ++ntl) {
-          const int i = (ntl * 8 + a) * 4 + 2 * ri;
-          const float2 z = __fmul2_rn(__fmul2_rn(f2(Z[i], Z[i + 1]), mtv[ntl]), f2(mcv, mcv));
-          Z[i] = z.x;
-          Z[i + 1] = z.y;
-          zlo = min3(zlo, z.x, z.y);
-          zhi = max3(zhi, z.x, z.y);
-        }
-      }
-  }
+    }
   const float zl = warp_min(zlo);
   const float zh = warp_max(zhi);
   if (lane == 0) {
-    sm.zmin[warp] = zl;
-    sm.zmax[warp] = zh;
+    sm.q.zmin[warp] = zl;
+    sm.q.zmax[warp] = zh;
   }
   __syncthreads();
-  const float zero = fminf(fminf(sm.zmin[0], sm.zmin[1]), fminf(sm.zmin[2], sm.zmin[3]));
-  const float zmx = fmaxf(fmaxf(sm.zmax[0], sm.zmax[1]), fmaxf(sm.zmax[2], sm.zmax[3]));
+  const float zero = fminf(fminf(sm.q.zmin[0], sm.q.zmin[1]), fminf(sm.q.zmin[2], sm.q.zmin[3]));
+  const float zmx = fmaxf(fmaxf(sm.q.zmax[0], sm.q.zmax[1]), fmaxf(sm.q.zmax[2], sm.q.zmax[3]));
   constexpr int LB = (1 << BITS) - 1;
   float step = __fdiv_rn(__fsub_rn(zmx, zero), static_cast<float>(LB));
   if (step == 0.f) step = 1.f;
@@ -539,18 +428,14 @@ __device__ __forceinline__ void quantize_tile(const TileOut& o, QuantScratch& sm
   for (int bl = 0; bl < 16; ++bl)
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      int idx;                             // index of the (h = 0) element; h = 1 is idx + 1
-      if (KL) {   // bl = ml*8 + a;  j = ri + 2*nb;  h = rj
-        const int ml = bl >> 3, a = bl & 7, nb = j >> 1, ri = j & 1;
-        idx = ((ml * 8 + a) * 2 + nb) * 4 + 2 * ri;
-      } else {    // V layout: bl = (ntl>>1)*8 + a;  j = ri + 2*(ntl&1);  h = rj
-        const int ntl = 2 * (bl >> 3) + (j >> 1), a = bl & 7, ri = j & 1;
-        idx = (ntl * 8 + a) * 4 + 2 * ri;
-      }
+      // index of the (h = 0) element, h = 1 is idx + 1; bl = (ntl>>1)*8 + a,
+      // j = ri + 2*(ntl&1), h = rj
+      const int ntl = 2 * (bl >> 3) + (j >> 1), a = bl & 7, ri = j & 1;
+      const int idx = (ntl * 8 + a) * 4 + 2 * ri;
       const float2 y = __ffma2_rn(f2(Z[idx], Z[idx + 1]), f2(inv, inv), f2(nzi, nzi));
       const float2 r = __fadd2_rn(y, f2(kMagic, kMagic));
       // 0 <= y <= 2^b - 1 up to rounding, so rne(y) sits in the low BITS bits of r
-      if (SIDE == 0 && !KL) {
+      if (SIDE == 0) {
         // K codes held in the V layout: this lane has (channel g, tokens 2c, 2c+1)
         // of an 8x8 block; the K fragment wants (token g, channels 2c, 2c+1).
         // One transpose of the block's 16-bit code pairs, then the K register
@@ -574,7 +459,7 @@ __device__ __forceinline__ void quantize_tile(const TileOut& o, QuantScratch& sm
     *reinterpret_cast<uint4*>(dst + ((warp * BITS + cc) * 32 + lane) * 16) = v4;
   }
   if (tid == 0) {
-    float* tailp = reinterpret_cast<float*>(sm.rec + 512);
+    float* tailp = reinterpret_cast<float*>(sm.q.rec + 512);
     tailp[0] = zero;
     tailp[1] = step;
     tailp[2] = 0.f;
@@ -582,7 +467,7 @@ __device__ __forceinline__ void quantize_tile(const TileOut& o, QuantScratch& sm
   }
   __syncthreads();
   if (tid < kScaleRec / 16) {
-    *reinterpret_cast<uint4*>(o.scales + tid * 16) = *reinterpret_cast<const uint4*>(sm.rec + tid * 16);
+    *reinterpret_cast<uint4*>(o.scales + tid * 16) = *reinterpret_cast<const uint4*>(sm.q.rec + tid * 16);
   }
 }
 
