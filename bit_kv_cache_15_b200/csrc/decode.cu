@@ -145,6 +145,9 @@ __device__ __noinline__ void quantize_full_tail(const DecodeArgs& p, uint8_t* sm
   o.iters = p.iters;
   if (side == 0) quantize_tile<0, KB, false>(o, sq, xs, 0u);
   else quantize_tile<1, VB, false>(o, sq, xs, 0u);
+  // order the generic-proxy accesses to the staged tile and the scratch before
+  // any later tile copy (async proxy) into the same shared memory
+  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
   __syncthreads();   // the staged tile and the scratch are free again
 }
 
@@ -888,6 +891,9 @@ __device__ __forceinline__ bool decode_segment(const DecodeArgs& p, uint8_t* sme
     }
     rec[4 + d] = a;
   }
+  // the merge area is dead: order its generic-proxy accesses before the next
+  // segment's tile copies (async proxy) into the same shared memory
+  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
   __syncthreads();   // the merge area and the q buffers are free for the next segment
   return !failed;
 }
