@@ -1205,12 +1205,20 @@ __global__ void __launch_bounds__(kDThreads, KVARN_D_MIN_CTAS) decode_kernel(con
 #pragma unroll 1
     for (int side = 0; side < 2; ++side)
       if (items & (2 << side)) quantize_full_tail<KB, VB>(p, smem, b, h, L, side);
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) sh_last = atomicAdd(p.counters + pair, sg_done) + sg_done == sg_nu;
+    __syncthreads();   // the CTA's record writes are ordered before thread 0's arrival
+    if (tid == 0) {
+      // one acquire-release add at GPU scope: releases this CTA's records (the
+      // barrier above puts them before it) and, for the last arrival, acquires
+      // every earlier CTA's; the barrier below passes that on to the CTA
+      int old;
+      asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;\n"
+                   : "=r"(old)
+                   : "l"(p.counters + pair), "r"(sg_done)
+                   : "memory");
+      sh_last = old + sg_done == sg_nu;
+    }
     __syncthreads();
     if (sh_last) {
-      __threadfence();
       combine_pair(p, b, h, grp, L, seq_valid(p, L), sg_pst, pair_tiles(L, seq_valid(p, L)), sh_W, P);
     }
   }
