@@ -203,9 +203,12 @@ def run_gpu(args):
     stream = torch.cuda.current_stream(dev)
 
     def step():
+        # NVTX: one range per step on a timeline (the library marks each of its calls too)
+        torch.cuda.nvtx.range_push("kvarn.step")
         K.quantize_tiles(k_app, v_app, slot_app, packed, scales, cfg, dev_status=status, stream=stream)
         K.decode_attention(q, packed, scales, tail, bt, sl, cfg, out=out, workspace=ws, dev_status=status,
                            stream=stream)
+        torch.cuda.nvtx.range_pop()
 
     for _ in range(args.warmup):
         step()

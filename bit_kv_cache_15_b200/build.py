@@ -10,6 +10,7 @@ import os
 import shutil
 import subprocess
 import sys
+from concurrent.futures import ThreadPoolExecutor
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
@@ -53,6 +54,12 @@ def up_to_date() -> bool:
 STALL_LIB = os.path.join(HERE, "libkvarn_stalltest.so")
 STALL_DEFINES = ["-DKVARN_TEST_STALL_FIRST_UNIT=1", "-DKVARN_WAIT_LIMIT_LOG2=10"]
 
+# The debug variant: the same kernels with their own index arithmetic checked
+# on the device (a failed check reports KVARN_DEV_INTERNAL and skips the
+# access).  Tests run it against the release library on the same inputs.
+DEBUG_LIB = os.path.join(HERE, "libkvarn_debug.so")
+DEBUG_DEFINES = ["-DKVARN_DEBUG=1"]
+
 
 def _compile(src: str, obj: str, defines, verbose: bool) -> None:
     cmd = [nvcc(), *NVCC_FLAGS, *defines, "-I", os.path.join(ROOT, "include"), "-c", os.path.join(CSRC, src),
@@ -84,19 +91,23 @@ def _fresh(lib: str) -> bool:
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and up_to_date() and _fresh(STALL_LIB):
+    if not force and up_to_date() and _fresh(STALL_LIB) and _fresh(DEBUG_LIB):
         return LIB
     objdir = os.path.join(HERE, "_build")
     os.makedirs(objdir, exist_ok=True)
-    objs = []
-    for src in SOURCES:
-        obj = os.path.join(objdir, src.replace(".cu", ".o"))
-        _compile(src, obj, [], verbose)
-        objs.append(obj)
-    _link(objs, LIB)
+    objs = [os.path.join(objdir, src.replace(".cu", ".o")) for src in SOURCES]
+    debug_objs = [os.path.join(objdir, src.replace(".cu", "_debug.o")) for src in SOURCES]
     stall_obj = os.path.join(objdir, "decode_stalltest.o")
-    _compile("decode.cu", stall_obj, STALL_DEFINES, verbose)
+    jobs = [(src, obj, []) for src, obj in zip(SOURCES, objs)]
+    jobs += [(src, obj, DEBUG_DEFINES) for src, obj in zip(SOURCES, debug_objs)]
+    jobs.append(("decode.cu", stall_obj, STALL_DEFINES))
+    # the nvcc runs are independent: run them side by side
+    with ThreadPoolExecutor(max_workers=min(len(jobs), os.cpu_count() or 1)) as ex:
+        for f in [ex.submit(_compile, src, obj, defines, verbose) for src, obj, defines in jobs]:
+            f.result()
+    _link(objs, LIB)
     _link([stall_obj if o.endswith(os.sep + "decode.o") else o for o in objs], STALL_LIB)
+    _link(debug_objs, DEBUG_LIB)
     return LIB
 
 

@@ -30,6 +30,24 @@ __device__ __forceinline__ void report_status(int32_t* st, int code) {
   if (st != nullptr) atomicCAS(st, 0, code);
 }
 
+// Debug builds (-DKVARN_DEBUG=1) check the kernels' own index arithmetic on
+// the device: a failed check reports KVARN_DEV_INTERNAL and the caller skips
+// the guarded access.  In release builds the check is the constant true and
+// compiles away.
+#ifndef KVARN_DEBUG
+#define KVARN_DEBUG 0
+#endif
+__device__ __forceinline__ bool debug_ok(bool cond, int32_t* st) {
+#if KVARN_DEBUG
+  if (!cond) report_status(st, KVARN_DEV_INTERNAL);
+  return cond;
+#else
+  (void)cond;
+  (void)st;
+  return true;
+#endif
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

@@ -186,7 +186,7 @@ __device__ void decode_tail(const DecodeArgs& p, uint8_t* smem, int b, int h, in
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g8 = lane >> 2, c = lane & 3;
   const int tl = (L & 127) + p.append;
-  if (tl == 0) return;
+  if (tl == 0 || !debug_ok(tl <= kTile, p.status)) return;
   const int pw = (b * p.Hkv + h) * p.ngrp + grp;   // work pair: (sequence, KV head, column group)
   const int nun = (tl + kTU - 1) / kTU;
   const __half* kt = p.tail + (((int64_t)b * 2 + 0) * p.Hkv + h) * (int64_t)(kTile * kHeadDim);
@@ -408,15 +408,17 @@ __device__ __forceinline__ int run_units(const DecodeArgs& p, uint8_t* stage_bas
   constexpr int U = T::U, MT = T::MT;
   const int lane = threadIdx.x & 31, g8 = lane >> 2, c = lane & 3;
   const int32_t* btab = p.block_table + (int64_t)b * p.max_blocks;
+  // block id of tile t of the sequence (debug builds: an index past the row reads as a bad block)
+  auto block_of = [&](int t) -> int32_t { return debug_ok(t >= 0 && t < p.max_blocks, p.status) ? btab[t] : -1; };
   // ok0 / ok1: the unit now in flight in stage 0 / 1 has a valid block
   bool ok0 = false, ok1 = false;
   if (n_mine > 0) {
-    const bool o = issue_unit<KB, VB>(p, stage_base, my_bars, kbase, u0, btab[t_begin + u0 / U], h, lane);
+    const bool o = issue_unit<KB, VB>(p, stage_base, my_bars, kbase, u0, block_of(t_begin + u0 / U), h, lane);
     if (kbase & 1) ok1 = o; else ok0 = o;
   }
   if (n_mine > 1) {
     const bool o = issue_unit<KB, VB>(p, stage_base, my_bars, kbase + 1, u0 + ustep,
-                                      btab[t_begin + (u0 + ustep) / U], h, lane);
+                                      block_of(t_begin + (u0 + ustep) / U), h, lane);
     if (kbase & 1) ok0 = o; else ok1 = o;
   }
   int k_fail = -1;
@@ -425,7 +427,7 @@ __device__ __forceinline__ int run_units(const DecodeArgs& p, uint8_t* stage_bas
     const int kg = kbase + k;
     const int stg = kg & 1;
     // block id of unit k + 2, loaded now so it is in hand when that copy is issued
-    const int32_t blk_next = k + 2 < n_mine ? btab[t_begin + (u0 + (k + 2) * ustep) / U] : 0;
+    const int32_t blk_next = k + 2 < n_mine ? block_of(t_begin + (u0 + (k + 2) * ustep) / U) : 0;
     if (!__all_sync(0xffffffffu, mbar_wait_bounded(&my_bars[stg], (kg >> 1) & 1))) {
       if (lane == 0) report_status(p.status, KVARN_DEV_TIMEOUT);
       k_fail = k;
@@ -994,6 +996,8 @@ __device__ void combine_columns(const DecodeArgs& p, int b, int h, int grp, int 
   // W >= P every CTA range is non-empty, so each of them wrote a record.
   const int i_lo = nt > 0 ? sk_owner(W, P, pst) : 0;
   const int n_rec = nt > 0 ? sk_owner(W, P, pst + nt - 1) - i_lo + 1 : 0;
+  // debug builds: the records read below are slots pair + i_lo .. pair + i_lo + n_rec - 1 of the workspace
+  if (!debug_ok(i_lo >= 0 && n_rec >= 0 && i_lo + n_rec <= P && P <= kDecodeMaxCtas, p.status)) return;
   const bool dense = W >= P;
   const bool has_tail = (L & 127) + p.append != 0;
   // a warp merges column slots warp and warp + 4 together, so one round of
@@ -1187,6 +1191,12 @@ __global__ void __launch_bounds__(kDThreads, KVARN_D_MIN_CTAS) decode_kernel(con
     const int sp = sg_h, L = sg_L, t_a = sg_ta, t_e = sg_te;
     const int h = sp / p.ngrp, grp = sp - (sp / p.ngrp) * p.ngrp;
     const int pair = b * p.Hkv * p.ngrp + sp;
+    // debug builds: the pair's record slot (pair + cta) and counter lie in the workspace
+    // (uniform across the CTA: every input is in shared memory or the launch)
+    if (!debug_ok(b < p.B && sp < p.Hkv * p.ngrp && cta < kDecodeMaxCtas, p.status)) {
+      ok = false;
+      continue;
+    }
     if (ok && t_a < t_e) {
       ok = decode_segment<KB, VB>(p, smem, b, h, grp, L, t_a, t_e, woff, rearm,
                                   p.ws + static_cast<int64_t>(pair + cta) * p.C * kPartialFloats);

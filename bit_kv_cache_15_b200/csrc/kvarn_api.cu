@@ -15,7 +15,28 @@
 #include "../../include/kvarn.h"
 #include "kvarn_internal.h"
 
+// NVTX ranges around every call that enqueues GPU work, so a timeline tool
+// shows which library call launched which kernels (header-only NVTX 3: with
+// no tool attached a range costs a null check).  -DKVARN_NVTX=0 removes them.
+#ifndef KVARN_NVTX
+#define KVARN_NVTX 1
+#endif
+#if KVARN_NVTX
+#include <nvtx3/nvToolsExt.h>
+#endif
+
 namespace {
+
+struct NvtxRange {
+#if KVARN_NVTX
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+#else
+  explicit NvtxRange(const char*) {}
+#endif
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 bool bits_ok(int b) { return b == 2 || b == 4 || b == 8; }
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -132,6 +153,7 @@ size_t kvarn_decode_workspace_bytes(const kvarn_config* cfg, const kvarn_decode_
 kvarn_status kvarn_quantize_tiles(const void* k, const void* v, const int64_t* slot_mapping, int64_t num_tokens,
                                   int32_t num_kv_heads, int64_t num_blocks, void* packed_cache, void* scales,
                                   const kvarn_config* cfg, int32_t* dev_status, void* stream) {
+  const NvtxRange nvtx_range("kvarn_quantize_tiles");
   return quantize_impl(k, v, slot_mapping, num_tokens, num_kv_heads, num_blocks, packed_cache, scales, cfg,
                        nullptr, dev_status, stream);
 }
@@ -140,6 +162,7 @@ kvarn_status kvarn_quantize_tiles_debug(const void* k, const void* v, const int6
                                         int64_t num_tokens, int32_t num_kv_heads, int64_t num_blocks,
                                         void* packed_cache, void* scales, const kvarn_config* cfg,
                                         float* debug_logscales, int32_t* dev_status, void* stream) {
+  const NvtxRange nvtx_range("kvarn_quantize_tiles_debug");
   if (debug_logscales == nullptr && num_tokens > 0) return KVARN_ERR_INVALID_ARGUMENT;
   return quantize_impl(k, v, slot_mapping, num_tokens, num_kv_heads, num_blocks, packed_cache, scales, cfg,
                        debug_logscales, dev_status, stream);
@@ -210,6 +233,7 @@ kvarn_status kvarn_decode_attention(const void* q, const void* packed_cache, con
                                     const void* fp16_tail, const int32_t* block_table, const int32_t* seq_lens,
                                     void* out, const kvarn_decode_dims* dims, const kvarn_config* cfg,
                                     void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream) {
+  const NvtxRange nvtx_range("kvarn_decode_attention");
   return decode_impl(q, nullptr, nullptr, packed_cache, scales, fp16_tail, block_table, seq_lens, out, dims, cfg,
                      workspace, workspace_bytes, dev_status, stream, 0, 1);
 }
@@ -226,6 +250,7 @@ kvarn_status kvarn_decode_attention_multiquery(const void* q, int32_t q_len, con
                                                const int32_t* seq_lens, void* out, const kvarn_decode_dims* dims,
                                                const kvarn_config* cfg, void* workspace, size_t workspace_bytes,
                                                int32_t* dev_status, void* stream) {
+  const NvtxRange nvtx_range("kvarn_decode_attention_multiquery");
   return decode_impl(q, nullptr, nullptr, packed_cache, scales, fp16_tail, block_table, seq_lens, out, dims, cfg,
                      workspace, workspace_bytes, dev_status, stream, 0, q_len);
 }
@@ -235,6 +260,7 @@ kvarn_status kvarn_decode_attention_append(const void* q, const void* k_new, con
                                            const int32_t* seq_lens, void* out, const kvarn_decode_dims* dims,
                                            const kvarn_config* cfg, void* workspace, size_t workspace_bytes,
                                            int32_t* dev_status, void* stream) {
+  const NvtxRange nvtx_range("kvarn_decode_attention_append");
   return decode_impl(q, k_new, v_new, packed_cache, scales, fp16_tail, block_table, seq_lens, out, dims, cfg,
                      workspace, workspace_bytes, dev_status, stream, 1, 1);
 }
@@ -243,6 +269,7 @@ kvarn_status kvarn_decode_attention_noalloc(const void* q, const void* packed_ca
                                             const void* fp16_tail, const int32_t* block_table,
                                             const int32_t* seq_lens, void* out, const kvarn_decode_dims* dims,
                                             const kvarn_config* cfg, int32_t* dev_status, void* stream) {
+  const NvtxRange nvtx_range("kvarn_decode_attention_noalloc");
   // Same path as kvarn_decode_attention, with the library's fixed device
   // scratch standing in for the caller's workspace.
   kvarn_status st = kvarn_config_validate(cfg);
@@ -311,6 +338,7 @@ kvarn_status kvarn_decode_attention_fp16(const void* q, const void* k_cache, con
                                          const int32_t* block_table, const int32_t* seq_lens, void* out,
                                          const kvarn_decode_dims* dims, float sm_scale, void* workspace,
                                          size_t workspace_bytes, int32_t* dev_status, void* stream) {
+  const NvtxRange nvtx_range("kvarn_decode_attention_fp16");
   return baseline_impl(q, k_cache, v_cache, block_table, seq_lens, out, dims, sm_scale, 1.f, 1.f, 0, workspace,
                        workspace_bytes, dev_status, stream);
 }
@@ -319,6 +347,7 @@ kvarn_status kvarn_decode_attention_fp8(const void* q, const void* k_cache, cons
                                         const int32_t* block_table, const int32_t* seq_lens, void* out,
                                         const kvarn_decode_dims* dims, float sm_scale, float k_scale, float v_scale,
                                         void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream) {
+  const NvtxRange nvtx_range("kvarn_decode_attention_fp8");
   return baseline_impl(q, k_cache, v_cache, block_table, seq_lens, out, dims, sm_scale, k_scale, v_scale, 1,
                        workspace, workspace_bytes, dev_status, stream);
 }

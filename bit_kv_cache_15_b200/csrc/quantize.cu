@@ -108,9 +108,13 @@ __global__ void __launch_bounds__(kQThreads, KVARN_Q_MIN_CTAS) quantize_kernel(c
       break;
     }
     // which paged block: slot_mapping[128 * grp] must start a block of the pool
-    const int64_t slot = p.slot_mapping[grp * kTile];
+    // debug builds: the tile's coordinates lie inside the input
+    const bool coords_ok = debug_ok(grp >= 0 && grp < p.num_groups && h >= 0 && h < p.hkv, p.status);
+    const int64_t slot = coords_ok ? p.slot_mapping[grp * kTile] : -1;
     const int64_t blk = slot >> 7;
-    if (slot < 0 || (slot & 127) != 0 || blk >= p.num_blocks) {
+    if (!coords_ok) {
+      // reported as KVARN_DEV_INTERNAL; nothing is written
+    } else if (slot < 0 || (slot & 127) != 0 || blk >= p.num_blocks) {
       if (tid == 0) report_status(p.status, KVARN_DEV_BAD_SLOT);
     } else {
       const uint32_t xs = smem_u32(sm.x[stage][0]);

@@ -73,6 +73,9 @@ typedef enum {
 #define KVARN_DEV_BAD_BLOCK 2      /* block_table entry beyond the pool */
 #define KVARN_DEV_BAD_SEQ_LEN 3    /* seq_len < 0 or > 128 * max_blocks_per_seq */
 #define KVARN_DEV_TIMEOUT 4        /* a bounded wait on an asynchronous copy gave up */
+#define KVARN_DEV_INTERNAL 5       /* debug builds (KVARN_DEBUG=1) only: one of the kernels' own
+                                      index checks failed, i.e. a library defect; the access it
+                                      guards was skipped, so the outputs of that call are invalid */
 
 typedef struct {
   int32_t version;         /* KVARN_ABI_VERSION */

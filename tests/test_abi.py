@@ -31,6 +31,16 @@ def test_every_declared_symbol_is_exported():
         assert n in K._SIGS, f"binding misses {n}"
 
 
+@pytest.mark.parametrize("path", [build.DEBUG_LIB, build.STALL_LIB])
+def test_test_builds_load_and_export_the_same_symbols(path):
+    """The debug build (device-side index checks) and the stall-test build
+    load on the host and export the same C ABI as the release library."""
+    lib = ctypes.CDLL(path)
+    for n in declared_functions():
+        assert hasattr(lib, n), (path, n)
+    assert lib.kvarn_abi_version() == K.lib.kvarn_abi_version()
+
+
 def test_abi_version_and_status_strings():
     assert K.lib.kvarn_abi_version() == 1
     assert K.lib.kvarn_status_string(0) == b"KVARN_OK"
