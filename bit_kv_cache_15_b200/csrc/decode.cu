@@ -16,11 +16,12 @@
 // cut into equal contiguous ranges, one per CTA of a grid of two CTAs per SM.
 // A CTA decodes each run of one pair's tiles in its range with all 4 warps
 // (units round-robin over the warps, each warp running its own online
-// softmax, merged into one partial record per query head), attends a tail
-// unit in its range exactly in the unrotated domain, and the last CTA to
-// finish a pair merges its records and applies H / 128.  Each warp streams
-// its tiles through a private 2-stage shared-memory ring filled by bulk
-// copies (cp.async.bulk on the TMA engine).  Codes are laid out in the mma
+// softmax, merged into one partial record per query head) and attends a
+// tail unit in its range exactly in the unrotated domain.  A second,
+// dependent grid (one CTA per pair, a programmatic dependent launch) merges
+// each pair's records and applies H / 128 once the decode grid has
+// completed.  Each warp streams its tiles through a private 2-stage
+// shared-memory ring filled by bulk copies (cp.async.bulk on the TMA engine).  Codes are laid out in the mma
 // fragment order, so a lane's 16-byte shared loads are its operands; each
 // masked code pair is already an f16x2 of exact subnormals.  Both
 // contractions run on the tensor cores (mma.m16n8k16, fp32 accumulate): K
@@ -988,6 +989,7 @@ __device__ void sk_locate(const DecodeArgs& p, int cta, int P, long long* W_out,
 // tail record from its own slot.  One warp per head; lane owns channels
 // 4*lane .. 4*lane + 3.  Records written by other CTAs are read with
 // ld.global.cg (L2), never through L1.
+template <int NC, int CH>
 __device__ void combine_columns(const DecodeArgs& p, int b, int h, int grp, int L, bool valid, long long pst, int nt,
                                 long long W, int P, int col0, int col1) {
   const int lane = threadIdx.x & 31;
@@ -1000,13 +1002,13 @@ __device__ void combine_columns(const DecodeArgs& p, int b, int h, int grp, int 
   if (!debug_ok(i_lo >= 0 && n_rec >= 0 && i_lo + n_rec <= P && P <= kDecodeMaxCtas, p.status)) return;
   const bool dense = W >= P;
   const bool has_tail = (L & 127) + p.append != 0;
-  // a warp merges column slots warp and warp + 4 together, so one round of
-  // L2 loads serves both
-  int gh[2];
-  bool hl[2];
-  int64_t orow[2];
+  // a warp merges NC column slots (col0, then col1) together, so one round of
+  // L2 loads serves them all; records are read CH at a time
+  int gh[NC];
+  bool hl[NC];
+  int64_t orow[NC];
 #pragma unroll
-  for (int k = 0; k < 2; ++k) {
+  for (int k = 0; k < NC; ++k) {
     int qi;
     gh[k] = k == 0 ? col0 : col1;
     hl[k] = col_row(p, b, h, grp, gh[k], &orow[k], &qi);
@@ -1014,18 +1016,20 @@ __device__ void combine_columns(const DecodeArgs& p, int b, int h, int grp, int 
   if (!hl[0]) return;
   if (!valid || L + p.append == 0) {
 #pragma unroll
-    for (int k = 0; k < 2; ++k)
+    for (int k = 0; k < NC; ++k)
       if (hl[k]) {
         __half* o = p.out + orow[k] + 4 * lane;
         *reinterpret_cast<uint2*>(o) = make_uint2(0u, 0u);
       }
     return;
   }
-  float M[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f}, a[2][4];
-  float mt[2], lt[2];
-  float4 vt[2];
+  float M[NC], l[NC], a[NC][4];
+  float mt[NC], lt[NC];
+  float4 vt[NC];
 #pragma unroll
-  for (int k = 0; k < 2; ++k) {
+  for (int k = 0; k < NC; ++k) {
+    M[k] = -INFINITY;
+    l[k] = 0.f;
 #pragma unroll
     for (int i = 0; i < 4; ++i) a[k][i] = 0.f;
     const float* trec = p.ws_tail + ((int64_t)pair * p.C + (hl[k] ? gh[k] : 0)) * kPartialFloats;
@@ -1034,17 +1038,16 @@ __device__ void combine_columns(const DecodeArgs& p, int b, int h, int grp, int 
     lt[k] = t ? __ldcg(trec + 1) : 0.f;
     vt[k] = t ? __ldcg(reinterpret_cast<const float4*>(trec + 4 + 4 * lane)) : make_float4(0.f, 0.f, 0.f, 0.f);
   }
-  constexpr int kChunk = 8;
-  for (int k0 = 0; k0 < n_rec; k0 += kChunk) {
-    float mr[2][kChunk], lr[2][kChunk];
-    float4 vr[2][kChunk];
+  for (int k0 = 0; k0 < n_rec; k0 += CH) {
+    float mr[NC][CH], lr[NC][CH];
+    float4 vr[NC][CH];
 #pragma unroll
-    for (int q = 0; q < kChunk; ++q) {
+    for (int q = 0; q < CH; ++q) {
       const int i = i_lo + k0 + q;
       bool live = k0 + q < n_rec;
       if (live && !dense) live = max(sk_begin(W, P, i), pst) < min(sk_begin(W, P, i + 1), pst + nt);
 #pragma unroll
-      for (int k = 0; k < 2; ++k) {
+      for (int k = 0; k < NC; ++k) {
         const bool lk = live && hl[k];
         const float* r = p.ws + ((int64_t)(pair + (lk ? i : i_lo)) * p.C + (hl[k] ? gh[k] : 0)) * kPartialFloats;
         mr[k][q] = lk ? __ldcg(r) : -INFINITY;
@@ -1053,9 +1056,9 @@ __device__ void combine_columns(const DecodeArgs& p, int b, int h, int grp, int 
       }
     }
 #pragma unroll
-    for (int q = 0; q < kChunk; ++q)
+    for (int q = 0; q < CH; ++q)
 #pragma unroll
-      for (int k = 0; k < 2; ++k) {
+      for (int k = 0; k < NC; ++k) {
         if (mr[k][q] == -INFINITY) continue;
         const float Mn = fmaxf(M[k], mr[k][q]);
         const float fo = ex2_fast(M[k] - Mn), fr = ex2_fast(mr[k][q] - Mn);
@@ -1068,7 +1071,7 @@ __device__ void combine_columns(const DecodeArgs& p, int b, int h, int grp, int 
       }
   }
 #pragma unroll
-  for (int k = 0; k < 2; ++k) {
+  for (int k = 0; k < NC; ++k) {
     if (!hl[k]) continue;
     float* ak = a[k];
     {   // acc H / 128
@@ -1103,29 +1106,32 @@ __device__ void combine_columns(const DecodeArgs& p, int b, int h, int grp, int 
   }
 }
 
-// The CTA version: warp w merges columns w and w + 4.
-__device__ __forceinline__ void combine_pair(const DecodeArgs& p, int b, int h, int grp, int L, bool valid,
-                                             long long pst, int nt, long long W, int P) {
+// Half a pair's columns by one CTA: warp w merges column 4 * half + w alone,
+// reading up to 16 records per round of L2 loads.
+__device__ __forceinline__ void combine_half(const DecodeArgs& p, int b, int h, int grp, int half, int L,
+                                             bool valid, long long pst, int nt, long long W, int P) {
   const int warp = threadIdx.x >> 5;
-  combine_columns(p, b, h, grp, L, valid, pst, nt, W, P, warp, warp + kDWarps);
+  combine_columns<1, 16>(p, b, h, grp, L, valid, pst, nt, W, P, kDWarps * half + warp, kMaxG);
 }
 
 // ------------------------------------------------------------------ main kernel
 
 // Stream-K: CTA `cta` of P walks its unit range [W*cta/P, W*(cta+1)/P) pair by
 // pair.  For each pair it meets it decodes the run of full tiles in its range
-// (one partial record per query head, slot pair + cta), attends the tail if
-// the pair's tail unit is in its range, then adds the number of units it did
-// to the pair's counter (cleared before the launch).  The CTA that brings the
-// counter to the pair's unit count merges the pair.  Nothing waits on anything.
+// (one partial record per query head, slot pair + cta) and attends the tail if
+// the pair's tail unit is in its range.  The pairs are merged by merge_kernel,
+// behind this grid.  No CTA waits on another.
 template <int KB, int VB>
 __global__ void __launch_bounds__(kDThreads, KVARN_D_MIN_CTAS) decode_kernel(const __grid_constant__ DecodeArgs p) {
   extern __shared__ __align__(128) uint8_t smem[];
   // walker state (thread 0) and the current segment, in shared memory so that
   // almost nothing of the walk is live in registers across a segment
-  __shared__ long long sh_W, sh_u, sh_ps, sg_pst;
-  __shared__ int sh_b, sg_b, sg_h, sg_L, sg_nu, sg_ta, sg_te, sg_done, sg_tail, sh_last;
+  __shared__ long long sh_W, sh_u, sh_ps;
+  __shared__ int sh_b, sg_b, sg_h, sg_L, sg_ta, sg_te, sg_tail;
   const int tid = threadIdx.x, cta = blockIdx.x, P = gridDim.x;
+  // the merge grid (launched behind this one) may start as CTAs of this grid
+  // exit; it waits for this grid's completion before reading any record
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
   if (tid < 32) {
     long long W, ps;
     int b0;
@@ -1164,8 +1170,6 @@ __global__ void __launch_bounds__(kDThreads, KVARN_D_MIN_CTAS) decode_kernel(con
         sg_b = b;
         sg_h = h;
         sg_L = L;
-        sg_nu = nu;
-        sg_pst = pst;
         sg_ta = static_cast<int>(u - pst);
         sg_te = static_cast<int>(min(e - pst, static_cast<long long>(pair_tiles(L, seq_valid(p, L)))));
         // last units of the work items after the tiles: tail attention, then
@@ -1180,7 +1184,6 @@ __global__ void __launch_bounds__(kDThreads, KVARN_D_MIN_CTAS) decode_kernel(con
           if (k < items && m >= u && m < e) flags |= 1 << k;
         }
         sg_tail = flags;
-        sg_done = static_cast<int>(e - u);
         sh_u = e;
       }
     }
@@ -1215,23 +1218,47 @@ __global__ void __launch_bounds__(kDThreads, KVARN_D_MIN_CTAS) decode_kernel(con
 #pragma unroll 1
     for (int side = 0; side < 2; ++side)
       if (items & (2 << side)) quantize_full_tail<KB, VB>(p, smem, b, h, L, side);
-    __syncthreads();   // the CTA's record writes are ordered before thread 0's arrival
-    if (tid == 0) {
-      // one acquire-release add at GPU scope: releases this CTA's records (the
-      // barrier above puts them before it) and, for the last arrival, acquires
-      // every earlier CTA's; the barrier below passes that on to the CTA
-      int old;
-      asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;\n"
-                   : "=r"(old)
-                   : "l"(p.counters + pair), "r"(sg_done)
-                   : "memory");
-      sh_last = old + sg_done == sg_nu;
+  }
+}
+
+// The merge (a10): two CTAs per work pair (sequence, KV head, column group),
+// one per half of its columns, launched behind the decode grid as a
+// programmatic dependent launch.  Its CTAs may become resident while the
+// decode grid still runs (as decode CTAs exit); each locates its pair's units
+// from seq_lens (an input), then waits in griddepcontrol.wait, which returns
+// once the decode grid has completed and its writes are visible, and merges
+// the pair's records.  P: the decode grid's CTA count (it fixes which CTAs
+// wrote records for the pair).
+__global__ void __launch_bounds__(kDThreads) merge_kernel(const __grid_constant__ DecodeArgs p, int P) {
+  __shared__ long long sh_W, sh_pst;
+  const int pair = blockIdx.x >> 1, half = blockIdx.x & 1;   // two CTAs per pair: column halves
+  const int per_seq = p.Hkv * p.ngrp;
+  const int b = pair / per_seq, sp = pair - (pair / per_seq) * per_seq;
+  const int h = sp / p.ngrp, grp = sp - (sp / p.ngrp) * p.ngrp;
+  const int L = p.seq_lens[b];
+  const bool valid = seq_valid(p, L);
+  if (threadIdx.x < 32) {   // total units W and the first unit of sequence b, by one warp
+    const int lane = threadIdx.x;
+    long long all = 0, before = 0;
+    for (int s = lane; s < p.B; s += 32) {
+      const int Ls = p.seq_lens[s];
+      const long long u = static_cast<long long>(pair_units(p, Ls, seq_valid(p, Ls))) * per_seq;
+      all += u;
+      if (s < b) before += u;
     }
-    __syncthreads();
-    if (sh_last) {
-      combine_pair(p, b, h, grp, L, seq_valid(p, L), sg_pst, pair_tiles(L, seq_valid(p, L)), sh_W, P);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      all += __shfl_xor_sync(0xffffffffu, all, o);
+      before += __shfl_xor_sync(0xffffffffu, before, o);
+    }
+    if (lane == 0) {
+      sh_W = all;
+      sh_pst = before + static_cast<long long>(sp) * pair_units(p, L, valid);
     }
   }
+  __syncthreads();
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");   // the decode grid's records are complete
+  combine_half(p, b, h, grp, half, L, valid, sh_pst, pair_tiles(L, valid), sh_W, P);
 }
 
 
@@ -1255,11 +1282,22 @@ cudaError_t launch_d(const DecodeArgs& p, cudaStream_t stream) {
     ctas[dev] = n < 1 ? 1 : (n > kDecodeMaxCtas ? kDecodeMaxCtas : n);
     configured.fetch_or(bit, std::memory_order_acq_rel);
   }
-  // the per-(seq, KV head) unit counters start every call at zero
-  cudaError_t e = cudaMemsetAsync(p.counters, 0, static_cast<size_t>(p.B) * p.Hkv * p.ngrp * sizeof(int), stream);
-  if (e != cudaSuccess) return e;
   decode_kernel<KB, VB><<<ctas[dev], kDThreads, T::kSmem, stream>>>(p);
-  return cudaGetLastError();
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int pairs = p.B * p.Hkv * p.ngrp;
+  if (pairs == 0) return cudaSuccess;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
+  cfg.blockDim = dim3(kDThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, merge_kernel, p, ctas[dev]);
 }
 
 }  // namespace
