@@ -1304,8 +1304,8 @@ cudaError_t launch_d(const DecodeArgs& p, cudaStream_t stream) {
 
 // ------------------------------------------------------------------ fixed scratch
 // Device-resident scratch for kvarn_decode_attention_noalloc: the stream-K
-// partial records and arrival counters live in this file-scope array instead
-// of a caller-supplied workspace.  Every GPU that loads the library holds these
+// partial records live in this file-scope array instead of a caller-supplied
+// workspace.  Every GPU that loads the library holds these
 // bytes until exit.  Its device address is looked up once per device ordinal
 // and cached for the life of the process: after a reset of the device's
 // primary context (cudaDeviceReset) the cached address is stale.

@@ -197,7 +197,7 @@ static kvarn_status decode_impl(const void* q, const void* k_new, const void* v_
   p.block_table = block_table;
   p.seq_lens = seq_lens;
   p.out = static_cast<__half*>(out);
-  {   // tile records, tail records, counters; per (sequence, KV head) the
+  {   // tile records, tail records, reserved words; per (sequence, KV head) the
       // G * q_len (query, head) columns form groups of up to 8
     const int cols = (dims->num_q_heads / dims->num_kv_heads) * q_len;
     p.qlen = q_len;

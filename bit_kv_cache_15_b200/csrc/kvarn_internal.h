@@ -37,7 +37,7 @@ struct DecodeArgs {
   __half* out;
   float* ws;            // tile partial records [(B * Hkv * ngrp + kDecodeMaxCtas) * C]
   float* ws_tail;       // tail partial records [B * Hkv * G]
-  int* counters;        // B * Hkv arrival counters (zeroed by each call)
+  int* counters;        // B * Hkv reserved words of the workspace (unused by the decode)
   int B, Hq, Hkv, G, max_blocks;
   int64_t num_blocks;
   int kb, vb;

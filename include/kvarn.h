@@ -114,10 +114,11 @@ KVARN_API size_t kvarn_scale_bytes_per_block(int32_t num_kv_heads);
 
 /* Bytes of decode workspace needed for these dims: 528-byte partial records
  * ((B*Hkv + 320) * G for runs of full tiles, B*Hkv*G for the fp16 tails;
- * 320 bounds the decode grid) followed by one int32 counter per (sequence,
- * KV head).  Depends only on cfg and dims (not on seq_lens, max_blocks or
- * the device).  Its contents need no initialisation: each call clears its
- * counters first. */
+ * 320 bounds the decode grid) followed by one reserved int32 word per
+ * (sequence, KV head).  Depends only on cfg and dims (not on seq_lens,
+ * max_blocks or the device).  Its contents need no initialisation: every
+ * record a call reads is written earlier in the same call (the decode grid
+ * writes the partial records, the merge grid launched behind it reads them). */
 KVARN_API size_t kvarn_decode_workspace_bytes(const kvarn_config* cfg, const kvarn_decode_dims* dims);
 
 /* Quantise-on-write of whole 128-token tiles ([hypho] 四步流水线 steps 1-4;
@@ -260,10 +261,8 @@ KVARN_API kvarn_status kvarn_decode_attention_multiquery(const void* q, int32_t 
  *    primary context is reset (cudaDeviceReset) the cached address is stale,
  *    so do not use this entry point across such a reset.
  *  - All calls on a device share the one array and it keeps the previous
- *    call's contents.  The only words that must start at zero are the
- *    per-(sequence, KV head) arrival counters, and each call clears them
- *    (cudaMemsetAsync on the array, no allocation) before its kernel runs;
- *    the partial records a call reads are written earlier in the same call.
+ *    call's contents; no word of it needs a starting value, because the
+ *    partial records a call reads are written earlier in the same call.
  *    Calls whose kernels overlap on the GPU (different streams, no ordering)
  *    race on the array; order them on one stream or by events.
  *  - It calls no cudaMalloc, cudaFree or other allocating routine. */

@@ -76,7 +76,7 @@ def test_noalloc_matches_workspace_entry_point_twice(K):
 def test_noalloc_rejects_problems_beyond_its_scratch(K):
     cfg = K.config("kvarn_k4v2_g128")
     # (B*Hkv + 320)*G tile records plus B*Hkv*G tail records of 528 B (and the
-    # counters) exceed the fixed 8 MiB array
+    # reserved words) exceed the fixed 8 MiB array
     d = K.dims(4096, 64, 8, 64, 4096)
     assert K.decode_workspace_bytes(cfg, d) > (8 << 20)
     one = torch.zeros(16, dtype=torch.uint8, device="cuda")
