@@ -333,9 +333,8 @@ def run_gpu(args):
                        "l2": f"inputs larger than L2: {(q_bytes + d_bytes) / 1e6:.0f} MB of algorithmic traffic per step"},
             "e2e": {"value": world * BATCH * args.steps / (ms_e2e * 1e-3), "unit": "decode tokens/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            # our kernels per step: quantize_kernel and decode_kernel (the decode's
-            # 256-byte counter clear is a cudaMemsetAsync, not one of our kernels)
-            "gpu_launches": 2 * args.steps,
+            # our kernels per step: quantize_kernel, decode_kernel and the decode's merge_kernel
+            "gpu_launches": 3 * args.steps,
             "roofline": roof,
             "kernels": {
                 "quantize": {"us": tq_ms * 1e3, "tiles_per_s": tiles / (tq_ms * 1e-3), "tflops": q_tflops,
