@@ -1055,20 +1055,37 @@ __device__ void combine_columns(const DecodeArgs& p, int b, int h, int grp, int 
         vr[k][q] = lk ? __ldcg(reinterpret_cast<const float4*>(r + 4 + 4 * lane)) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
     }
+    // the round's records at once: their max, then the weights 2^(m - max)
+    // (independent) and the weighted sums in four interleaved partials, so no
+    // step waits on the previous record; rounds combine online
 #pragma unroll
-    for (int q = 0; q < CH; ++q)
+    for (int k = 0; k < NC; ++k) {
+      float Mr = -INFINITY;
 #pragma unroll
-      for (int k = 0; k < NC; ++k) {
-        if (mr[k][q] == -INFINITY) continue;
-        const float Mn = fmaxf(M[k], mr[k][q]);
-        const float fo = ex2_fast(M[k] - Mn), fr = ex2_fast(mr[k][q] - Mn);
-        l[k] = fmaf(l[k], fo, lr[k][q] * fr);
-        a[k][0] = fmaf(a[k][0], fo, vr[k][q].x * fr);
-        a[k][1] = fmaf(a[k][1], fo, vr[k][q].y * fr);
-        a[k][2] = fmaf(a[k][2], fo, vr[k][q].z * fr);
-        a[k][3] = fmaf(a[k][3], fo, vr[k][q].w * fr);
-        M[k] = Mn;
+      for (int q = 0; q < CH; ++q) Mr = fmaxf(Mr, mr[k][q]);
+      if (Mr == -INFINITY) continue;   // no live record in this round
+      float lp[4] = {0.f, 0.f, 0.f, 0.f};
+      float4 ap[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) ap[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int q = 0; q < CH; ++q) {
+        const float f = mr[k][q] == -INFINITY ? 0.f : ex2_fast(mr[k][q] - Mr);
+        lp[q & 3] = fmaf(f, lr[k][q], lp[q & 3]);
+        ap[q & 3].x = fmaf(f, vr[k][q].x, ap[q & 3].x);
+        ap[q & 3].y = fmaf(f, vr[k][q].y, ap[q & 3].y);
+        ap[q & 3].z = fmaf(f, vr[k][q].z, ap[q & 3].z);
+        ap[q & 3].w = fmaf(f, vr[k][q].w, ap[q & 3].w);
       }
+      const float Mn = fmaxf(M[k], Mr);
+      const float fo = ex2_fast(M[k] - Mn), fr = ex2_fast(Mr - Mn);
+      l[k] = fmaf(l[k], fo, ((lp[0] + lp[1]) + (lp[2] + lp[3])) * fr);
+      a[k][0] = fmaf(a[k][0], fo, ((ap[0].x + ap[1].x) + (ap[2].x + ap[3].x)) * fr);
+      a[k][1] = fmaf(a[k][1], fo, ((ap[0].y + ap[1].y) + (ap[2].y + ap[3].y)) * fr);
+      a[k][2] = fmaf(a[k][2], fo, ((ap[0].z + ap[1].z) + (ap[2].z + ap[3].z)) * fr);
+      a[k][3] = fmaf(a[k][3], fo, ((ap[0].w + ap[1].w) + (ap[2].w + ap[3].w)) * fr);
+      M[k] = Mn;
+    }
   }
 #pragma unroll
   for (int k = 0; k < NC; ++k) {
