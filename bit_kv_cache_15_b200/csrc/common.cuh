@@ -8,7 +8,10 @@
 #pragma once
 
 #include <cuda_fp16.h>
+#include <cuda_runtime.h>
 #include <stdint.h>
+
+#include <utility>
 
 #include "../../include/kvarn.h"
 
@@ -25,6 +28,28 @@ constexpr float kLog2e = 1.4426950408889634f;
 #define KVARN_WAIT_LIMIT_LOG2 26
 #endif
 constexpr uint32_t kWaitLimit = 1u << KVARN_WAIT_LIMIT_LOG2;
+
+// Launch a kernel as a programmatic dependent launch: its CTAs may become
+// resident while the previous kernel in the stream still runs (once that
+// kernel's CTAs have all issued griddepcontrol.launch_dependents or exited).
+// Every kernel launched this way issues griddepcontrol.wait before its first
+// global-memory access, which returns once the previous kernel has completed
+// and its writes are visible, so ordering against any predecessor holds.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                              Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 __device__ __forceinline__ void report_status(int32_t* st, int code) {
   if (st != nullptr) atomicCAS(st, 0, code);

@@ -1147,8 +1147,11 @@ __global__ void __launch_bounds__(kDThreads, KVARN_D_MIN_CTAS) decode_kernel(con
   __shared__ int sh_b, sg_b, sg_h, sg_L, sg_ta, sg_te, sg_tail;
   const int tid = threadIdx.x, cta = blockIdx.x, P = gridDim.x;
   // the merge grid (launched behind this one) may start as CTAs of this grid
-  // exit; it waits for this grid's completion before reading any record
+  // exit; it waits for this grid's completion before reading any record.
+  // This grid is itself a programmatic dependent launch: it waits for the
+  // previous kernel in the stream before its first global-memory access.
   asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
   if (tid < 32) {
     long long W, ps;
     int b0;
@@ -1248,6 +1251,8 @@ __global__ void __launch_bounds__(kDThreads, KVARN_D_MIN_CTAS) decode_kernel(con
 // wrote records for the pair).
 __global__ void __launch_bounds__(kDThreads) merge_kernel(const __grid_constant__ DecodeArgs p, int P) {
   __shared__ long long sh_W, sh_pst;
+  // the next kernel in the stream may become resident as these CTAs exit
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
   const int pair = blockIdx.x >> 1, half = blockIdx.x & 1;   // two CTAs per pair: column halves
   const int per_seq = p.Hkv * p.ngrp;
   const int b = pair / per_seq, sp = pair - (pair / per_seq) * per_seq;
@@ -1299,22 +1304,12 @@ cudaError_t launch_d(const DecodeArgs& p, cudaStream_t stream) {
     ctas[dev] = n < 1 ? 1 : (n > kDecodeMaxCtas ? kDecodeMaxCtas : n);
     configured.fetch_or(bit, std::memory_order_acq_rel);
   }
-  decode_kernel<KB, VB><<<ctas[dev], kDThreads, T::kSmem, stream>>>(p);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(decode_kernel<KB, VB>, dim3(ctas[dev]), dim3(kDThreads), static_cast<size_t>(T::kSmem),
+                             stream, p);
   if (e != cudaSuccess) return e;
   const int pairs = p.B * p.Hkv * p.ngrp;
   if (pairs == 0) return cudaSuccess;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
-  cfg.blockDim = dim3(kDThreads);
-  cfg.dynamicSmemBytes = 0;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, merge_kernel, p, ctas[dev]);
+  return launch_pdl(merge_kernel, dim3(static_cast<unsigned>(2 * pairs)), dim3(kDThreads), 0, stream, p, ctas[dev]);
 }
 
 }  // namespace
