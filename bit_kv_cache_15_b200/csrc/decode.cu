@@ -504,10 +504,10 @@ __device__ __forceinline__ int run_units(const DecodeArgs& p, uint8_t* stage_bas
         const float2 f01 = __half22float2(h01), f89 = __half22float2(h89);
         const __half2 l01 = __floats2half2_rn(x0 - f01.x, x1 - f01.y);
         const __half2 l89 = __floats2half2_rn(x8 - f89.x, x9 - f89.y);
-        {   // sum of exactly the q' values the mma sees (hi + lo)
-          const float2 g01 = __half22float2(l01), g89 = __half22float2(l89);
-          qsum += ((f01.x + g01.x) + (f01.y + g01.y)) + ((f89.x + g89.x) + (f89.y + g89.y));
-        }
+        // sum of q' for the zero-point term, from the fp32 values: hi + lo
+        // carries them to about 2^-22, so the mma's q' and this sum differ by
+        // a score offset far below the fp16 output rounding
+        qsum += (x0 + x1) + (x8 + x9);
         qb0[kt] = h2_as_u32(h01);
         qb1[kt] = h2_as_u32(h89);
         ql0[kt] = h2_as_u32(l01);
