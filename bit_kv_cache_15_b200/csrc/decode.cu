@@ -1146,11 +1146,8 @@ __global__ void __launch_bounds__(kDThreads, KVARN_D_MIN_CTAS) decode_kernel(con
   __shared__ long long sh_W, sh_u, sh_ps;
   __shared__ int sh_b, sg_b, sg_h, sg_L, sg_ta, sg_te, sg_tail;
   const int tid = threadIdx.x, cta = blockIdx.x, P = gridDim.x;
-  // the merge grid (launched behind this one) may start as CTAs of this grid
-  // exit; it waits for this grid's completion before reading any record.
-  // This grid is itself a programmatic dependent launch: it waits for the
-  // previous kernel in the stream before its first global-memory access.
-  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+  // This grid is a programmatic dependent launch: it waits for the previous
+  // kernel in the stream before its first global-memory access.
   asm volatile("griddepcontrol.wait;\n" ::: "memory");
   if (tid < 32) {
     long long W, ps;
@@ -1239,6 +1236,11 @@ __global__ void __launch_bounds__(kDThreads, KVARN_D_MIN_CTAS) decode_kernel(con
     for (int side = 0; side < 2; ++side)
       if (items & (2 << side)) quantize_full_tail<KB, VB>(p, smem, b, h, L, side);
   }
+  // the merge grid behind this one may launch once every CTA of this grid has
+  // reached here (it waits for this grid's completion before reading any
+  // record).  Triggering at the start instead let merge CTAs sit resident
+  // beside running decode CTAs, which cost the quantise + decode step 7 us.
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
 }
 
 // The merge (a10): two CTAs per work pair (sequence, KV head, column group),
