@@ -1253,8 +1253,6 @@ __global__ void __launch_bounds__(kDThreads, KVARN_D_MIN_CTAS) decode_kernel(con
 // wrote records for the pair).
 __global__ void __launch_bounds__(kDThreads) merge_kernel(const __grid_constant__ DecodeArgs p, int P) {
   __shared__ long long sh_W, sh_pst;
-  // the next kernel in the stream may become resident as these CTAs exit
-  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
   const int pair = blockIdx.x >> 1, half = blockIdx.x & 1;   // two CTAs per pair: column halves
   const int per_seq = p.Hkv * p.ngrp;
   const int b = pair / per_seq, sp = pair - (pair / per_seq) * per_seq;

@@ -79,6 +79,11 @@ __global__ void __launch_bounds__(kQThreads, KVARN_Q_MIN_CTAS) quantize_kernel(c
   tmem_fence_before_sync();
   __syncthreads();
   tmem_fence_after_sync();
+  // a programmatic dependent launch: the setup above may overlap the previous
+  // kernel in the stream; wait for it before the first global-memory access.
+  // No early launch_dependents: the next kernel launches as these CTAs exit
+  // (waiting CTAs resident beside running ones slowed the step by 10-20 us).
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
   int64_t id = blockIdx.x;
   if (id < total && tid == 0) {
     int side, h;
@@ -221,8 +226,7 @@ cudaError_t launch_q(const QuantArgs& p, cudaStream_t stream) {
   const int64_t tiles = 2 * p.num_groups * p.hkv;
   const int64_t slots = static_cast<int64_t>(sms[dev]) * ctas_per_sm[dev];
   const unsigned grid = static_cast<unsigned>(tiles < slots ? tiles : slots);
-  quantize_kernel<KB, VB><<<grid, kQThreads, smem, stream>>>(mk, mv, p);
-  return cudaGetLastError();
+  return launch_pdl(quantize_kernel<KB, VB>, dim3(grid), dim3(kQThreads), static_cast<size_t>(smem), stream, mk, mv, p);
 }
 
 }  // namespace
