@@ -1245,12 +1245,14 @@ __global__ void __launch_bounds__(kDThreads, KVARN_D_MIN_CTAS) decode_kernel(con
 
 // The merge (a10): two CTAs per work pair (sequence, KV head, column group),
 // one per half of its columns, launched behind the decode grid as a
-// programmatic dependent launch.  Its CTAs may become resident while the
-// decode grid still runs (as decode CTAs exit); each locates its pair's units
-// from seq_lens (an input), then waits in griddepcontrol.wait, which returns
-// once the decode grid has completed and its writes are visible, and merges
-// the pair's records.  P: the decode grid's CTA count (it fixes which CTAs
-// wrote records for the pair).
+// programmatic dependent launch.  Its CTAs may become resident once every
+// decode CTA has finished its range (the decode's trigger), before the decode
+// grid has fully drained; each locates its pair's units from seq_lens (an
+// input of the decode call, written before the decode grid started), then
+// waits in griddepcontrol.wait, which returns once the decode grid has
+// completed and its writes are visible, and merges the pair's records.
+// P: the decode grid's CTA count (it fixes which CTAs wrote records for the
+// pair).
 __global__ void __launch_bounds__(kDThreads) merge_kernel(const __grid_constant__ DecodeArgs p, int P) {
   __shared__ long long sh_W, sh_pst;
   const int pair = blockIdx.x >> 1, half = blockIdx.x & 1;   // two CTAs per pair: column halves
