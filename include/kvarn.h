@@ -20,6 +20,12 @@
  *    allocates no memory and keeps no state between calls.
  *  - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
  *    stream) and the call returns without synchronising.  Calls are reentrant.
+ *  - The kernels are programmatic dependent launches: a kernel's CTAs may
+ *    become resident before the previous kernel in the stream has finished
+ *    and do their on-chip set-up, but each waits for that kernel's completion
+ *    (griddepcontrol.wait) before its first global-memory access, so stream
+ *    order holds against any earlier work.  They work inside CUDA graph
+ *    capture as well.
  *  - Each kernel's launch set-up (its shared-memory attribute and grid size)
  *    is done once per device ordinal (ordinals 0-63; others get
  *    KVARN_ERR_CUDA) and kept for the process; a reset of the device's primary
