@@ -1211,7 +1211,7 @@ __global__ void __launch_bounds__(kDThreads, KVARN_D_MIN_CTAS) decode_kernel(con
     const int sp = sg_h, L = sg_L, t_a = sg_ta, t_e = sg_te;
     const int h = sp / p.ngrp, grp = sp - (sp / p.ngrp) * p.ngrp;
     const int pair = b * p.Hkv * p.ngrp + sp;
-    // debug builds: the pair's record slot (pair + cta) and counter lie in the workspace
+    // debug builds: the pair's record slot (pair + cta) lies in the workspace
     // (uniform across the CTA: every input is in shared memory or the launch)
     if (!debug_ok(b < p.B && sp < p.Hkv * p.ngrp && cta < kDecodeMaxCtas, p.status)) {
       ok = false;
@@ -1377,8 +1377,9 @@ size_t decode_workspace(int B, int Hq, int Hkv, int qlen) {
   const size_t C = cols < kMaxG ? cols : kMaxG;                           // records per column group
   const size_t pairs = static_cast<size_t>(B) * Hkv * ngrp;
   const size_t records = (pairs + kDecodeMaxCtas) * C + pairs * C;       // tile records, then tail records
-  const size_t counters = (pairs * sizeof(int32_t) + 15) & ~static_cast<size_t>(15);
-  return records * kPartialFloats * sizeof(float) + counters;
+  // then one reserved int32 word per work pair (kept so the size formula is stable)
+  const size_t reserved = (pairs * sizeof(int32_t) + 15) & ~static_cast<size_t>(15);
+  return records * kPartialFloats * sizeof(float) + reserved;
 }
 
 cudaError_t launch_decode(const DecodeArgs& p, cudaStream_t stream) {
