@@ -1,8 +1,8 @@
 """The debug build of the library (libkvarn_debug.so, built beside libkvarn.so
 with -DKVARN_DEBUG=1): the same kernels with their own index arithmetic
-checked on the device -- block-table rows, record slots and counters of the
-decode's work split, the merge's record range, the tail staging, the
-quantiser's tile coordinates.  A failed check would report KVARN_DEV_INTERNAL
+checked on the device -- block-table rows and record slots of the decode's
+work split, the merge's record range, the tail staging, the quantiser's tile
+coordinates.  A failed check would report KVARN_DEV_INTERNAL
 (5) and skip the guarded access; it never traps.
 
 On valid inputs no check may fire (the status stays 0), and every output must
