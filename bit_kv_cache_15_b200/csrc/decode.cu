@@ -18,12 +18,13 @@
 // (units round-robin over the warps, each warp running its own online
 // softmax, merged into one partial record per query head) and attends a
 // tail unit in its range exactly in the unrotated domain.  A second,
-// dependent grid (one CTA per pair, a programmatic dependent launch) merges
+// dependent grid (two CTAs per pair, a programmatic dependent launch) merges
 // each pair's records and applies H / 128 once the decode grid has
 // completed.  Each warp streams its tiles through a private 2-stage
-// shared-memory ring filled by bulk copies (cp.async.bulk on the TMA engine).  Codes are laid out in the mma
-// fragment order, so a lane's 16-byte shared loads are its operands; each
-// masked code pair is already an f16x2 of exact subnormals.  Both
+// shared-memory ring filled by bulk copies (cp.async.bulk on the TMA engine).
+// Codes are laid out in the mma fragment order, so a lane's 16-byte shared
+// loads are its operands; each masked code pair is already an f16x2 of exact
+// subnormals.  Both
 // contractions run on the tensor cores (mma.m16n8k16, fp32 accumulate): K
 // side rows = tokens, N = the 8 query heads; V side rows = channels, N =
 // heads, with the softmax weights moved from accumulator to operand layout
