@@ -379,8 +379,9 @@ __device__ __forceinline__ bool issue_unit(const DecodeArgs& p, uint8_t* stage_b
     if (ok) {
       const uint8_t* cb = p.packed + ((int64_t)blk * p.Hkv + h) * T::kCode;
       mbar_arrive_expect_tx(bar, T::kStage);
-      bulk_g2s(dst, cb + part * T::kUnitK, T::kUnitK, bar);
-      bulk_g2s(dst + T::kUnitK, cb + T::kCodeK + part * T::kUnitV, T::kUnitV, bar);
+      const uint64_t pol = l2_evict_first_policy();   // the codes are read once per call
+      bulk_g2s_hint(dst, cb + part * T::kUnitK, T::kUnitK, bar, pol);
+      bulk_g2s_hint(dst + T::kUnitK, cb + T::kCodeK + part * T::kUnitV, T::kUnitV, bar, pol);
       bulk_g2s(dst + T::kUnitK + T::kUnitV, p.scales + ((int64_t)blk * p.Hkv + h) * (2 * kScaleRec), 2 * kScaleRec,
                bar);
     } else {

@@ -40,12 +40,13 @@ constexpr int kMaxCtasPerSm = 512 / kTmemCols;
 __device__ __forceinline__ void load_tile(const CUtensorMap* map, uint8_t* dst, uint64_t* bar, int h, int64_t grp) {
   mbar_arrive_expect_tx(bar, 2 * kBox);
   const int t0 = static_cast<int>(grp * kTile);
+  const uint64_t pol = l2_evict_first_policy();   // the fp16 input is read once
 #pragma unroll
   for (int half = 0; half < 2; ++half) {
     asm volatile(
-        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3, %4}], [%5];\n" ::"r"(smem_u32(dst + half * kBox)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(64 * half), "r"(h), "r"(t0), "r"(smem_u32(bar))
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3, %4}], [%5], %6;\n" ::"r"(smem_u32(dst + half * kBox)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(64 * half), "r"(h), "r"(t0), "r"(smem_u32(bar)), "l"(pol)
         : "memory");
   }
 }
