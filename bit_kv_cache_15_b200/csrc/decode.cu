@@ -140,13 +140,13 @@ __device__ __noinline__ void quantize_full_tail(const DecodeArgs& p, uint8_t* sm
   for (int c16 = 0; c16 < 16; ++c16) cp_async16(xs + xoff(tid, c16), row + c16, 16);
   cp_async_wait_all();
   __syncthreads();
-  TileOut o;
-  o.codes = p.packed_w + ((int64_t)blk * p.Hkv + h) * (int64_t)(2048 * (KB + VB)) + (side == 0 ? 0 : 2048 * KB);
-  o.scales = p.scales_w + (((int64_t)blk * p.Hkv + h) * 2 + side) * (int64_t)kScaleRec;
-  o.dbg = nullptr;
-  o.iters = p.iters;
-  if (side == 0) quantize_tile<0, KB, false>(o, sq, xs, 0u);
-  else quantize_tile<1, VB, false>(o, sq, xs, 0u);
+  if (tid == 0) {   // read inside quantize_tile after its first barrier
+    sq.out.codes = p.packed_w + ((int64_t)blk * p.Hkv + h) * (int64_t)(2048 * (KB + VB)) + (side == 0 ? 0 : 2048 * KB);
+    sq.out.scales = p.scales_w + (((int64_t)blk * p.Hkv + h) * 2 + side) * (int64_t)kScaleRec;
+    sq.out.dbg = nullptr;
+  }
+  if (side == 0) quantize_tile<0, KB, false>(p.iters, sq, xs, 0u);
+  else quantize_tile<1, VB, false>(p.iters, sq, xs, 0u);
   // order the generic-proxy accesses to the staged tile and the scratch before
   // any later tile copy (async proxy) into the same shared memory
   asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");

@@ -20,8 +20,9 @@
 // The rotation uses H16 as the mma A operand and X as the B operand, so after
 // stage 2 each lane holds exactly the elements of the decode kernel's V-side
 // mma fragments (rows channels): V codes are packed in registers with no
-// cross-lane traffic, and K codes (rows tokens) after one movmatrix transpose
-// per 8x8 block of code pairs.
+// cross-lane traffic, and K codes (rows tokens) are packed the same way and
+// then moved to the K fragment order by one movmatrix transpose per packed
+// 32-bit word.
 // Used by the quantise-on-write kernel and by the decode kernel's append path.
 #pragma once
 #include "common.cuh"
@@ -45,6 +46,13 @@ constexpr int kXchStride = kHeadDim + 4;
 constexpr int kTokStride = 32 + 4;
 static_assert(8 * kTokStride <= 4 * kXchStride, "token exchange inside the warp's channel rows");
 
+// Where one tile's results go.
+struct TileOut {
+  uint8_t* codes;        // this side's code block (2048 * BITS bytes, 16-byte aligned)
+  uint8_t* scales;       // this side's 528-byte scale record
+  float* dbg;            // nullable: fp32 log-scales before rounding (256 floats)
+};
+
 // Per-CTA scratch of one tile's normalisation and quantisation.  Channels are
 // kept in the permuted order j = g*16 + 2a + ri of channel 16a + g + 8ri (the
 // order in which a lane of the register layout holds its 16 channels).
@@ -63,6 +71,10 @@ struct QuantScratch {
   };
   alignas(16) float u[kHeadDim];         // channel weights 2^(-2 lc), permuted order
   alignas(16) float wb[4][32];           // per-warp token-weight exchange
+  // Where the tile's results go, written by the caller's thread 0 before
+  // quantize_tile and read only after the tile's first CTA barrier: kept here
+  // rather than in registers, beside the 128 that hold R^2 during the passes.
+  TileOut out;
 };
 
 // channel of permuted index j = g*16 + 2a + ri
@@ -227,21 +239,15 @@ __device__ __forceinline__ void rotate_v(uint32_t xs, int warp, int lane, float 
 
 // ---------------------------------------------------------------- the tile
 
-// Where one tile's results go.
-struct TileOut {
-  uint8_t* codes;        // this side's code block (2048 * BITS bytes, 16-byte aligned)
-  uint8_t* scales;       // this side's 528-byte scale record
-  float* dbg;            // nullable: fp32 log-scales before rounding (256 floats)
-  int iters;
-};
-
 // Stages 2-5 for the fp16 tile staged at shared address xs (xoff layout), by
-// all 128 threads of the CTA.  STASH: keep R in tensor memory at tmem (this
-// CTA's allocation) between the rotation and quantisation; otherwise the
-// rotation is run a second time from the staged tile (same arithmetic).
+// all 128 threads of the CTA, with `iters` normalisation iterations; results go
+// where sm.out says.  STASH: keep R in tensor memory at tmem (this CTA's
+// allocation) between the rotation and quantisation; otherwise the rotation is
+// run a second time from the staged tile (same arithmetic).
 template <int SIDE, int BITS, bool STASH>
-__device__ __forceinline__ void quantize_tile(const TileOut& o, QuantScratch& sm, uint32_t xs, uint32_t tmem) {
+__device__ __forceinline__ void quantize_tile(int iters, QuantScratch& sm, uint32_t xs, uint32_t tmem) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const TileOut& o = sm.out;
   const int g = lane >> 2, c = lane & 3;
 
   // ---- 2. rotate
@@ -268,7 +274,7 @@ __device__ __forceinline__ void quantize_tile(const TileOut& o, QuantScratch& sm
   for (int i = 0; i < NT; ++i) wt[i] = 1.f;
   float lt_sum = 1.f, lc_sum = 1.f;   // this thread's token / channel sums of the last pass
 
-  for (int it = 0; it < o.iters; ++it) {
+  for (int it = 0; it < iters; ++it) {
     // channel pass: partial sums over this thread's 8 tokens for its 16
     // channels, to row (warp, c) of the exchange in the permuted order (four
     // 16-byte stores); thread j then sums permuted channel j over the 16 rows
@@ -306,30 +312,28 @@ __device__ __forceinline__ void quantize_tile(const TileOut& o, QuantScratch& sm
     }
     __syncthreads();
 
-    // token pass
+    // token pass: one accumulator per token pair, the 16 channel weights read
+    // in two halves of 8
     {
-      float uu[16];
+      float2 acc[4] = {f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f)};   // index ntl
 #pragma unroll
-      for (int k4 = 0; k4 < 4; ++k4) {
-        const float4 x = *reinterpret_cast<const float4*>(&sm.u[g * 16 + 4 * k4]);
-        uu[4 * k4] = x.x; uu[4 * k4 + 1] = x.y; uu[4 * k4 + 2] = x.z; uu[4 * k4 + 3] = x.w;
-      }
-      float s[8];    // index ntl*2 + rj
+      for (int hf = 0; hf < 2; ++hf) {
+        float uu[8];   // permuted positions 8*hf .. 8*hf+7 of this lane's 16: a = 4*hf + (k >> 1), ri = k & 1
 #pragma unroll
-      for (int ntl = 0; ntl < 4; ++ntl) {
-        float2 acc[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};   // 2 chains for ILP
+        for (int k4 = 0; k4 < 2; ++k4) {
+          const float4 x = *reinterpret_cast<const float4*>(&sm.u[g * 16 + 8 * hf + 4 * k4]);
+          uu[4 * k4] = x.x; uu[4 * k4 + 1] = x.y; uu[4 * k4 + 2] = x.z; uu[4 * k4 + 3] = x.w;
+        }
 #pragma unroll
-        for (int a = 0; a < 8; ++a)
+        for (int k = 0; k < 8; ++k)
 #pragma unroll
-          for (int ri = 0; ri < 2; ++ri) {
+          for (int ntl = 0; ntl < 4; ++ntl) {
+            const int a = 4 * hf + (k >> 1), ri = k & 1;
             const int i = (ntl * 8 + a) * 4 + 2 * ri;
-            const float uv = uu[a * 2 + ri];
-            acc[ri] = __ffma2_rn(f2(A[i], A[i + 1]), f2(uv, uv), acc[ri]);
+            acc[ntl] = __ffma2_rn(f2(A[i], A[i + 1]), f2(uu[k], uu[k]), acc[ntl]);
           }
-        const float2 t = __fadd2_rn(acc[0], acc[1]);
-        s[ntl * 2] = t.x;
-        s[ntl * 2 + 1] = t.y;
       }
+      const float s[8] = {acc[0].x, acc[0].y, acc[1].x, acc[1].y, acc[2].x, acc[2].y, acc[3].x, acc[3].y};   // index ntl*2 + rj
       // the 8 lanes g = 0..7 of one c hold partials of the same 8 tokens: row
       // g, columns c*8 .. c*8+7 of this warp's own exchange rows (free until
       // its next channel pass); lane (g, c) then sums column c*8 + g, i.e.
@@ -437,19 +441,28 @@ __device__ __forceinline__ void quantize_tile(const TileOut& o, QuantScratch& sm
       // 0 <= y <= 2^b - 1 up to rounding, so rne(y) sits in the low BITS bits of r
       if (SIDE == 0) {
         // K codes held in the V layout: this lane has (channel g, tokens 2c, 2c+1)
-        // of an 8x8 block; the K fragment wants (token g, channels 2c, 2c+1).
-        // One transpose of the block's 16-bit code pairs, then the K register
-        // j' = (token half) + 2 (channel half) = (j >> 1) + 2 (j & 1).
-        const uint32_t pr = __byte_perm(__float_as_uint(r.x), __float_as_uint(r.y), 0x5410);
-        const uint32_t tr = movmatrix_t(pr);
+        // of an 8x8 block; the K fragment wants (token g, channels 2c, 2c+1),
+        // in K register j' = (token half) + 2 (channel half) = (j >> 1) + 2 (j & 1).
+        // The codes go to their K-word bit fields here and each word is
+        // transposed once below.
         const int rk = 4 * bl + (j >> 1) + 2 * (j & 1);
-        words[rk / PER] |= (tr & static_cast<uint32_t>(LB | (LB << 16))) << (BITS * (rk % PER));
+        words[rk / PER] = bfi(__float_as_uint(r.x), words[rk / PER], BITS * (rk % PER), BITS);
+        words[rk / PER] = bfi(__float_as_uint(r.y), words[rk / PER], BITS * (rk % PER) + 16, BITS);
       } else {
         const int rho = 4 * bl + j;
         words[rho / PER] = bfi(__float_as_uint(r.x), words[rho / PER], BITS * (rho % PER), BITS);
         words[rho / PER] = bfi(__float_as_uint(r.y), words[rho / PER], BITS * (rho % PER) + 16, BITS);
       }
     }
+
+  if (SIDE == 0) {
+    // The transpose of an 8x8 block of 16-bit elements moves every element by
+    // the same lane permutation, whatever block it belongs to, so one
+    // transpose per word carries all the code fields packed into it (up to 8
+    // blocks' worth) to their K-fragment lanes and halves.
+#pragma unroll
+    for (int i = 0; i < NW; ++i) words[i] = movmatrix_t(words[i]);
+  }
 
   // ---- 5. store codes (16-byte chunks, lane-interleaved) and the scale record
   uint8_t* dst = o.codes;

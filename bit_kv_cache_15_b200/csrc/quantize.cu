@@ -30,6 +30,7 @@ struct QuantSmem {
   QuantScratch s;
   alignas(8) uint64_t bar[2];
   uint32_t tmem;                         // tensor-memory base of this CTA's R stash
+  int it_slot[kQThreads];                // per thread: the index of its next tile iteration
 };
 
 // A CTA allocates kTmemCols tensor-memory columns once; at most kMaxCtasPerSm
@@ -77,6 +78,7 @@ __global__ void __launch_bounds__(kQThreads, KVARN_Q_MIN_CTAS) quantize_kernel(c
     fence_barrier_init();
   }
   if (tid < 32) tmem_alloc(&sm.tmem);
+  sm.it_slot[tid] = 0;
   tmem_fence_before_sync();
   __syncthreads();
   tmem_fence_after_sync();
@@ -85,14 +87,20 @@ __global__ void __launch_bounds__(kQThreads, KVARN_Q_MIN_CTAS) quantize_kernel(c
   // No early launch_dependents: the next kernel launches as these CTAs exit
   // (waiting CTAs resident beside running ones slowed the step by 10-20 us).
   asm volatile("griddepcontrol.wait;\n" ::: "memory");
-  int64_t id = blockIdx.x;
-  if (id < total && tid == 0) {
+  if (blockIdx.x < total && tid == 0) {
     int side, h;
     int64_t grp;
-    tile_coords(p, id, side, grp, h);
+    tile_coords(p, blockIdx.x, side, grp, h);
     load_tile(side ? &map_v : &map_k, sm.x[0][0], &sm.bar[0], h, grp);
   }
-  for (int it = 0; id < total; ++it, id += gridDim.x) {
+  for (;;) {
+    // The iteration index goes through shared memory (each thread its own
+    // word), so that no loop state stays live in registers across the tile,
+    // whose passes need all but a few of them.
+    const int it = sm.it_slot[tid];
+    sm.it_slot[tid] = it + 1;
+    const int64_t id = blockIdx.x + static_cast<int64_t>(it) * gridDim.x;
+    if (id >= total) break;
     const int stage = it & 1;
     const int64_t nxt = id + gridDim.x;
     if (nxt < total && tid == 0) {   // the other stage was released at the end of the previous tile
@@ -124,13 +132,14 @@ __global__ void __launch_bounds__(kQThreads, KVARN_Q_MIN_CTAS) quantize_kernel(c
       if (tid == 0) report_status(p.status, KVARN_DEV_BAD_SLOT);
     } else {
       const uint32_t xs = smem_u32(sm.x[stage][0]);
-      TileOut o;
-      o.codes = p.packed + (blk * p.hkv + h) * (int64_t)(2048 * (p.kb + p.vb)) + (side == 0 ? 0 : 2048 * p.kb);
-      o.scales = p.scales + ((blk * p.hkv + h) * 2 + side) * (int64_t)kScaleRec;
-      o.dbg = p.dbg != nullptr ? p.dbg + ((grp * p.hkv + h) * 2 + side) * 256 : nullptr;
-      o.iters = p.iters;
-      if (side == 0) quantize_tile<0, KB, true>(o, sm.s, xs, sm.tmem);
-      else quantize_tile<1, VB, true>(o, sm.s, xs, sm.tmem);
+      if (tid == 0) {   // read inside quantize_tile after its first barrier
+        TileOut& o = sm.s.out;
+        o.codes = p.packed + (blk * p.hkv + h) * (int64_t)(2048 * (p.kb + p.vb)) + (side == 0 ? 0 : 2048 * p.kb);
+        o.scales = p.scales + ((blk * p.hkv + h) * 2 + side) * (int64_t)kScaleRec;
+        o.dbg = p.dbg != nullptr ? p.dbg + ((grp * p.hkv + h) * 2 + side) * 256 : nullptr;
+      }
+      if (side == 0) quantize_tile<0, KB, true>(p.iters, sm.s, xs, sm.tmem);
+      else quantize_tile<1, VB, true>(p.iters, sm.s, xs, sm.tmem);
     }
     __syncthreads();   // stage `stage` and the shared scratch are free again
   }
