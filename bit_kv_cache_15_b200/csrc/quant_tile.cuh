@@ -66,7 +66,6 @@ struct QuantScratch {
       float mt[kTile];                     // fp32(2^-Lt)
       float mc[kHeadDim];                  // fp32(2^-Lc)
       float zmin[4], zmax[4];
-      alignas(16) uint8_t rec[kScaleRec];  // staged scale record
     } q;
   };
   alignas(16) float u[kHeadDim];         // channel weights 2^(-2 lc), permuted order
@@ -369,8 +368,10 @@ __device__ __forceinline__ void quantize_tile(int iters, QuantScratch& sm, uint3
   const __half Lc16 = __float2half_rn(lc_own);
   sm.q.mt[t_own] = __double2float_rn(exp2(-static_cast<double>(__half2float(Lt16))));
   sm.q.mc[c_own] = __double2float_rn(exp2(-static_cast<double>(__half2float(Lc16))));
-  reinterpret_cast<__half*>(sm.q.rec)[t_own] = Lt16;
-  reinterpret_cast<__half*>(sm.q.rec + 256)[c_own] = Lc16;
+  // the scale record's log-scales, straight from the threads that own them
+  // (a warp's token scales fill one 64-byte run)
+  reinterpret_cast<__half*>(o.scales)[t_own] = Lt16;
+  reinterpret_cast<__half*>(o.scales + 256)[c_own] = Lc16;
   if (o.dbg != nullptr) {
     o.dbg[t_own] = lt_own;
     o.dbg[128 + c_own] = lc_own;
@@ -471,17 +472,7 @@ __device__ __forceinline__ void quantize_tile(int iters, QuantScratch& sm, uint3
     const uint4 v4 = make_uint4(words[4 * cc], words[4 * cc + 1], words[4 * cc + 2], words[4 * cc + 3]);
     *reinterpret_cast<uint4*>(dst + ((warp * BITS + cc) * 32 + lane) * 16) = v4;
   }
-  if (tid == 0) {
-    float* tailp = reinterpret_cast<float*>(sm.q.rec + 512);
-    tailp[0] = zero;
-    tailp[1] = step;
-    tailp[2] = 0.f;
-    tailp[3] = 0.f;
-  }
-  __syncthreads();
-  if (tid < kScaleRec / 16) {
-    *reinterpret_cast<uint4*>(o.scales + tid * 16) = *reinterpret_cast<const uint4*>(sm.q.rec + tid * 16);
-  }
+  if (tid == 0) *reinterpret_cast<float4*>(o.scales + 512) = make_float4(zero, step, 0.f, 0.f);
 }
 
 }  // namespace qt

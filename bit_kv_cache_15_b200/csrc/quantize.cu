@@ -31,7 +31,14 @@ struct QuantSmem {
   alignas(8) uint64_t bar[2];
   uint32_t tmem;                         // tensor-memory base of this CTA's R stash
   int it_slot[kQThreads];                // per thread: the index of its next tile iteration
+  alignas(8) int64_t slot[2];            // [stage] slot_mapping of the tile's first token
 };
+
+// 8-byte asynchronous copy global -> shared (through L1), in its own commit group
+__device__ __forceinline__ void fetch_slot(int64_t* dst, const int64_t* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;\n" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+  asm volatile("cp.async.commit_group;\n" ::: "memory");
+}
 
 // A CTA allocates kTmemCols tensor-memory columns once; at most kMaxCtasPerSm
 // CTAs share an SM's 512 columns, so the allocation never waits.
@@ -92,6 +99,7 @@ __global__ void __launch_bounds__(kQThreads, KVARN_Q_MIN_CTAS) quantize_kernel(c
     int64_t grp;
     tile_coords(p, blockIdx.x, side, grp, h);
     load_tile(side ? &map_v : &map_k, sm.x[0][0], &sm.bar[0], h, grp);
+    fetch_slot(&sm.slot[0], p.slot_mapping + grp * kTile);
   }
   for (;;) {
     // The iteration index goes through shared memory (each thread its own
@@ -108,6 +116,13 @@ __global__ void __launch_bounds__(kQThreads, KVARN_Q_MIN_CTAS) quantize_kernel(c
       int64_t grp;
       tile_coords(p, nxt, side, grp, h);
       load_tile(side ? &map_v : &map_k, sm.x[stage ^ 1][0], &sm.bar[stage ^ 1], h, grp);
+      fetch_slot(&sm.slot[stage ^ 1], p.slot_mapping + grp * kTile);
+    }
+    // thread 0: this tile's slot (fetched a tile ago) has landed; the barrier
+    // below publishes it to the CTA
+    if (tid == 0) {
+      if (nxt < total) asm volatile("cp.async.wait_group 1;\n" ::: "memory");
+      else asm volatile("cp.async.wait_group 0;\n" ::: "memory");
     }
     int side, h;
     int64_t grp;
@@ -124,7 +139,7 @@ __global__ void __launch_bounds__(kQThreads, KVARN_Q_MIN_CTAS) quantize_kernel(c
     // which paged block: slot_mapping[128 * grp] must start a block of the pool
     // debug builds: the tile's coordinates lie inside the input
     const bool coords_ok = debug_ok(grp >= 0 && grp < p.num_groups && h >= 0 && h < p.hkv, p.status);
-    const int64_t slot = coords_ok ? p.slot_mapping[grp * kTile] : -1;
+    const int64_t slot = coords_ok ? sm.slot[stage] : -1;
     const int64_t blk = slot >> 7;
     if (!coords_ok) {
       // reported as KVARN_DEV_INTERNAL; nothing is written
@@ -144,6 +159,7 @@ __global__ void __launch_bounds__(kQThreads, KVARN_Q_MIN_CTAS) quantize_kernel(c
     __syncthreads();   // stage `stage` and the shared scratch are free again
   }
   // every path reaches here with the CTA converged (the timeout break is CTA-uniform)
+  if (tid == 0) cp_async_wait_all();   // no slot copy outlives the CTA
   tmem_fence_before_sync();
   __syncthreads();
   tmem_fence_after_sync();
