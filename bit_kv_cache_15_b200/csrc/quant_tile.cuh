@@ -145,11 +145,14 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
   return r;
 }
 
-// insert the low `len` bits of x into y at bit `pos`
-__device__ __forceinline__ uint32_t bfi(uint32_t x, uint32_t y, int pos, int len) {
-  uint32_t r;
-  asm("bfi.b32 %0, %1, %2, %3, %4;\n" : "=r"(r) : "r"(x), "r"(y), "r"(pos), "r"(len));
-  return r;
+// The codes of a pair from their magic-add floats (1.5 * 2^23 + rne(y)): the
+// magic constant's low 16 bits are 0 and rne(y) lies in [0, 2^BITS - 1] (y is
+// (Z - zero) / step of the tile's own min and max, off by rounding errors far
+// below 1/2), so the low 16 bits of each float are its code and one byte
+// permute gives code.x | code.y << 16, ready to be shifted into its field of a
+// packed word (the fields do not overlap, so adding them is or-ing them).
+__device__ __forceinline__ uint32_t pair_codes(float2 r) {
+  return __byte_perm(__float_as_uint(r.x), __float_as_uint(r.y), 0x5410);
 }
 
 // ------------------------------------------------------------ tensor memory
@@ -278,23 +281,22 @@ __device__ __forceinline__ void quantize_tile(int iters, QuantScratch& sm, uint3
     // channels, to row (warp, c) of the exchange in the permuted order (four
     // 16-byte stores); thread j then sums permuted channel j over the 16 rows
     {
-      float s[16];   // index a*2 + ri = permuted position within this lane's 16
-#pragma unroll
-      for (int a = 0; a < 8; ++a)
-#pragma unroll
-        for (int ri = 0; ri < 2; ++ri) {
-          float2 acc = f2(0.f, 0.f);
-#pragma unroll
-          for (int ntl = 0; ntl < 4; ++ntl) {
-            const int i = (ntl * 8 + a) * 4 + 2 * ri;
-            acc = __ffma2_rn(f2(A[i], A[i + 1]), f2(wt[ntl * 2], wt[ntl * 2 + 1]), acc);
-          }
-          s[a * 2 + ri] = acc.x + acc.y;
-        }
       float* row = sm.xch + (warp * 4 + c) * kXchStride + g * 16;
 #pragma unroll
-      for (int k4 = 0; k4 < 4; ++k4)
-        *reinterpret_cast<float4*>(row + 4 * k4) = make_float4(s[4 * k4], s[4 * k4 + 1], s[4 * k4 + 2], s[4 * k4 + 3]);
+      for (int k4 = 0; k4 < 4; ++k4) {
+        // permuted positions 4*k4 .. 4*k4+3 (a = 2*k4 + (m >> 1), ri = m & 1):
+        // four independent chains, interleaved token group by token group
+        float2 acc[4] = {f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f)};
+#pragma unroll
+        for (int ntl = 0; ntl < 4; ++ntl)
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            const int i = (ntl * 8 + 2 * k4 + (m >> 1)) * 4 + 2 * (m & 1);
+            acc[m] = __ffma2_rn(f2(A[i], A[i + 1]), f2(wt[ntl * 2], wt[ntl * 2 + 1]), acc[m]);
+          }
+        *reinterpret_cast<float4*>(row + 4 * k4) =
+            make_float4(acc[0].x + acc[0].y, acc[1].x + acc[1].y, acc[2].x + acc[2].y, acc[3].x + acc[3].y);
+      }
     }
     __syncthreads();
     {
@@ -447,12 +449,10 @@ __device__ __forceinline__ void quantize_tile(int iters, QuantScratch& sm, uint3
         // The codes go to their K-word bit fields here and each word is
         // transposed once below.
         const int rk = 4 * bl + (j >> 1) + 2 * (j & 1);
-        words[rk / PER] = bfi(__float_as_uint(r.x), words[rk / PER], BITS * (rk % PER), BITS);
-        words[rk / PER] = bfi(__float_as_uint(r.y), words[rk / PER], BITS * (rk % PER) + 16, BITS);
+        words[rk / PER] += pair_codes(r) << (BITS * (rk % PER));
       } else {
         const int rho = 4 * bl + j;
-        words[rho / PER] = bfi(__float_as_uint(r.x), words[rho / PER], BITS * (rho % PER), BITS);
-        words[rho / PER] = bfi(__float_as_uint(r.y), words[rho / PER], BITS * (rho % PER) + 16, BITS);
+        words[rho / PER] += pair_codes(r) << (BITS * (rho % PER));
       }
     }
 

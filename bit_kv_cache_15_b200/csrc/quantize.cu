@@ -32,6 +32,10 @@ struct QuantSmem {
   uint32_t tmem;                         // tensor-memory base of this CTA's R stash
   int it_slot[kQThreads];                // per thread: the index of its next tile iteration
   alignas(8) int64_t slot[2];            // [stage] slot_mapping of the tile's first token
+  struct {
+    int64_t grp;
+    int side, h;
+  } coord[2];                            // [stage] the tile's coordinates (written by thread 0)
 };
 
 // 8-byte asynchronous copy global -> shared (through L1), in its own commit group
@@ -100,6 +104,9 @@ __global__ void __launch_bounds__(kQThreads, KVARN_Q_MIN_CTAS) quantize_kernel(c
     tile_coords(p, blockIdx.x, side, grp, h);
     load_tile(side ? &map_v : &map_k, sm.x[0][0], &sm.bar[0], h, grp);
     fetch_slot(&sm.slot[0], p.slot_mapping + grp * kTile);
+    sm.coord[0].grp = grp;
+    sm.coord[0].side = side;
+    sm.coord[0].h = h;
   }
   for (;;) {
     // The iteration index goes through shared memory (each thread its own
@@ -117,6 +124,9 @@ __global__ void __launch_bounds__(kQThreads, KVARN_Q_MIN_CTAS) quantize_kernel(c
       tile_coords(p, nxt, side, grp, h);
       load_tile(side ? &map_v : &map_k, sm.x[stage ^ 1][0], &sm.bar[stage ^ 1], h, grp);
       fetch_slot(&sm.slot[stage ^ 1], p.slot_mapping + grp * kTile);
+      sm.coord[stage ^ 1].grp = grp;
+      sm.coord[stage ^ 1].side = side;
+      sm.coord[stage ^ 1].h = h;
     }
     // thread 0: this tile's slot (fetched a tile ago) has landed; the barrier
     // below publishes it to the CTA
@@ -124,9 +134,6 @@ __global__ void __launch_bounds__(kQThreads, KVARN_Q_MIN_CTAS) quantize_kernel(c
       if (nxt < total) asm volatile("cp.async.wait_group 1;\n" ::: "memory");
       else asm volatile("cp.async.wait_group 0;\n" ::: "memory");
     }
-    int side, h;
-    int64_t grp;
-    tile_coords(p, id, side, grp, h);
     // every thread polls; the CTA proceeds only if all saw the copy land
     const bool landed = __syncthreads_and(mbar_wait_bounded(&sm.bar[stage], (it >> 1) & 1)) != 0;
     if (!landed) {
@@ -136,6 +143,9 @@ __global__ void __launch_bounds__(kQThreads, KVARN_Q_MIN_CTAS) quantize_kernel(c
       if (nxt < total) (void)mbar_wait_bounded(&sm.bar[stage ^ 1], ((it + 1) >> 1) & 1);
       break;
     }
+    // the tile's coordinates and slot, published by the barrier above
+    const int side = sm.coord[stage].side, h = sm.coord[stage].h;
+    const int64_t grp = sm.coord[stage].grp;
     // which paged block: slot_mapping[128 * grp] must start a block of the pool
     // debug builds: the tile's coordinates lie inside the input
     const bool coords_ok = debug_ok(grp >= 0 && grp < p.num_groups && h >= 0 && h < p.hkv, p.status);
