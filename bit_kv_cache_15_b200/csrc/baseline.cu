@@ -13,7 +13,11 @@
 // 2-stage ring filled by the TMA engine (128-byte swizzle), mma.m16n8k16 for
 // q.K (A = K rows via ldmatrix) and P.V (A = V^T via ldmatrix.trans), online
 // softmax per warp, merge per CTA, and the last CTA of a (seq, KV head)
-// combines the splits.  e4m3 tiles are widened to fp16 in shared memory.
+// combines the splits.  e4m3 tiles go to the tensor cores straight from the
+// staged bytes: ldmatrix of 8x8 blocks of byte pairs, widened to fp16 in
+// registers (cvt.rn.f16x2.e4m3x2), with the k and m orders of the MMAs
+// permuted to match (q is loaded in the same k order, and the output
+// channels are mapped back when the warps merge).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -35,8 +39,7 @@ template <int FP8>
 struct BaseTraits {
   // fp16: stage = K (2 boxes) + V (2 boxes); fp8: stage = K row tile + V row tile (128 B rows)
   static constexpr int kRaw = FP8 ? 2 * kUnit * 128 : 4 * kHalf16;
-  static constexpr int kConv = FP8 ? 4 * kHalf16 : 0;   // widened fp16 K, V (one buffer per warp)
-  static constexpr int kWarpBytes = 2 * kRaw + kConv;
+  static constexpr int kWarpBytes = 2 * kRaw;
   static constexpr int kBarOff = kBWarps * kWarpBytes;
   static constexpr int kSmem = kBarOff + 64;
 };
@@ -50,6 +53,10 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t x) {
   uint32_t y;
   asm("cvt.rn.f16x2.e4m3x2 %0, %1;\n" : "=r"(y) : "h"(x));
   return y;
+}
+// bytes (i, j) of x as an e4m3 pair (byte i to the low half)
+__device__ __forceinline__ uint32_t e4m3_bytes_to_f16x2(uint32_t x, unsigned sel) {
+  return e4m3x2_to_f16x2(static_cast<uint16_t>(__byte_perm(x, 0u, sel)));
 }
 
 __device__ __forceinline__ void tma_3d(const CUtensorMap* map, void* dst, uint64_t* bar, int c0, int c1, int c2) {
@@ -83,14 +90,18 @@ __device__ void baseline_split(const BaselineArgs& p, const CUtensorMap* mk, con
   }
   __syncwarp();
 
-  // q fragments (B operand of q.K): b0b1 = q[g8][16kt + 2c .. +1], b1 = +8; heads >= G are 0
+  // q fragments (B operand of q.K), heads >= G are 0.  fp16: b0 = q[g8][16kt +
+  // 2c .. +1], b1 = +8.  fp8: the k slots 2c, 2c+1, 2c+8, 2c+9 of block kt
+  // are channels 16kt + 4c .. 4c+3 (the order the e4m3 K fragments arrive in)
   uint32_t qb0[8], qb1[8];
   {
     const __half* qp = p.q + ((int64_t)b * p.Hq + h * G + g8) * kHeadDim;
 #pragma unroll
     for (int kt = 0; kt < 8; ++kt) {
-      qb0[kt] = g8 < G ? *reinterpret_cast<const uint32_t*>(qp + 16 * kt + 2 * c) : 0u;
-      qb1[kt] = g8 < G ? *reinterpret_cast<const uint32_t*>(qp + 16 * kt + 2 * c + 8) : 0u;
+      const int c0 = FP8 ? 16 * kt + 4 * c : 16 * kt + 2 * c;
+      const int c1 = FP8 ? c0 + 2 : c0 + 8;
+      qb0[kt] = g8 < G ? *reinterpret_cast<const uint32_t*>(qp + c0) : 0u;
+      qb1[kt] = g8 < G ? *reinterpret_cast<const uint32_t*>(qp + c1) : 0u;
     }
   }
   const float sl = p.sm_scale * kLog2e * (FP8 ? p.k_scale : 1.f);
@@ -149,59 +160,42 @@ __device__ void baseline_split(const BaselineArgs& p, const CUtensorMap* mk, con
     const int tok0 = tok_begin + (warp + k * kBWarps) * kUnit;
     const int valid_rows = min(kUnit, L - tok0);          // rows >= valid_rows are past the sequence
     uint8_t* raw = wbase + stg * T::kRaw;
-    uint8_t* kt16;
-    uint8_t* vt16;
-    if (FP8) {
-      // widen both 16 x 128 e4m3 tiles to the swizzled fp16 layout; zero rows past the sequence
-      uint8_t* conv = wbase + 2 * T::kRaw;
-#pragma unroll
-      for (int side = 0; side < 2; ++side) {
-        const uint8_t* src = raw + side * kUnit * 128;
-        uint8_t* dst = conv + side * 2 * kHalf16;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int idx = i * 32 + lane;                 // 128 chunks of 16 bytes
-          const int row = idx >> 3, c16 = idx & 7;       // fp8 row has 8 chunks of 16 channels
-          const uint4 v = *reinterpret_cast<const uint4*>(src + row * 128 + ((c16 ^ (row & 7)) << 4));
-          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-          uint32_t hx[8];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            hx[2 * j] = e4m3x2_to_f16x2(static_cast<uint16_t>(w[j] & 0xffffu));
-            hx[2 * j + 1] = e4m3x2_to_f16x2(static_cast<uint16_t>(w[j] >> 16));
-          }
-          const bool live = row < valid_rows;
-          const uint4 lo = live ? make_uint4(hx[0], hx[1], hx[2], hx[3]) : make_uint4(0, 0, 0, 0);
-          const uint4 hi = live ? make_uint4(hx[4], hx[5], hx[6], hx[7]) : make_uint4(0, 0, 0, 0);
-          *reinterpret_cast<uint4*>(dst + off16(row, 2 * c16)) = lo;
-          *reinterpret_cast<uint4*>(dst + off16(row, 2 * c16 + 1)) = hi;
-        }
+    if (!FP8 && valid_rows < kUnit) {   // zero V rows past the sequence (cache memory there is arbitrary)
+      uint8_t* vt16 = raw + 2 * kHalf16;
+      for (int idx = lane; idx < kUnit * 16; idx += 32) {
+        const int row = idx >> 4, c16 = idx & 15;
+        if (row >= valid_rows) *reinterpret_cast<uint4*>(vt16 + off16(row, c16)) = make_uint4(0, 0, 0, 0);
       }
       __syncwarp();
-      kt16 = conv;
-      vt16 = conv + 2 * kHalf16;
-    } else {
-      kt16 = raw;
-      vt16 = raw + 2 * kHalf16;
-      if (valid_rows < kUnit) {   // zero V rows past the sequence (cache memory there is arbitrary)
-        for (int idx = lane; idx < kUnit * 16; idx += 32) {
-          const int row = idx >> 4, c16 = idx & 15;
-          if (row >= valid_rows) *reinterpret_cast<uint4*>(vt16 + off16(row, c16)) = make_uint4(0, 0, 0, 0);
-        }
-        __syncwarp();
-      }
     }
     if (ok) {
       // q.K: 16 tokens x 8 heads, K = 128 channels
       float S[4] = {0.f, 0.f, 0.f, 0.f};
-      const uint32_t kb = smem_u32(kt16), vb = smem_u32(vt16);
       const int mi = lane >> 3;
-      const int arow = (lane & 7) + 8 * (mi & 1);
+      if (FP8) {
+        // 8x8 blocks of byte pairs: lanes 0-15 address rows 0-15 of chunk kt,
+        // lanes 16-31 of chunk kt + 1; a thread gets channels 4c .. 4c+3 of
+        // rows g8 and g8 + 8 of each chunk
+        const uint32_t kb8 = smem_u32(raw);
+        const int lrow = (lane & 7) + 8 * (mi & 1);
 #pragma unroll
-      for (int kt = 0; kt < 8; ++kt) {
-        uint32_t a0, a1, a2, a3;
-        ldmatrix_x4(kb + off16(arow, 2 * kt + (mi >> 1)), a0, a1, a2, a3);
-        mma_f16(S, a0, a1, a2, a3, qb0[kt], qb1[kt]);
+        for (int kt = 0; kt < 8; kt += 2) {
+          uint32_t r0, r1, r2, r3;
+          ldmatrix_x4(kb8 + lrow * 128 + (((kt + (mi >> 1)) ^ (lrow & 7)) << 4), r0, r1, r2, r3);
+          mma_f16(S, e4m3_bytes_to_f16x2(r0, 0x10), e4m3_bytes_to_f16x2(r1, 0x10), e4m3_bytes_to_f16x2(r0, 0x32),
+                  e4m3_bytes_to_f16x2(r1, 0x32), qb0[kt], qb1[kt]);
+          mma_f16(S, e4m3_bytes_to_f16x2(r2, 0x10), e4m3_bytes_to_f16x2(r3, 0x10), e4m3_bytes_to_f16x2(r2, 0x32),
+                  e4m3_bytes_to_f16x2(r3, 0x32), qb0[kt + 1], qb1[kt + 1]);
+        }
+      } else {
+        const uint32_t kb = smem_u32(raw);
+        const int arow = (lane & 7) + 8 * (mi & 1);
+#pragma unroll
+        for (int kt = 0; kt < 8; ++kt) {
+          uint32_t a0, a1, a2, a3;
+          ldmatrix_x4(kb + off16(arow, 2 * kt + (mi >> 1)), a0, a1, a2, a3);
+          mma_f16(S, a0, a1, a2, a3, qb0[kt], qb1[kt]);
+        }
       }
       // rows g8 and g8 + 8, heads 2c, 2c+1; log2 units; mask tokens past the sequence
       const bool v0 = g8 < valid_rows, v1 = g8 + 8 < valid_rows;
@@ -225,19 +219,49 @@ __device__ void baseline_split(const BaselineArgs& p, const CUtensorMap* mk, con
       lsum[1] = lsum[1] * al1 + (p1 + p3);
       const uint32_t bv0 = movmatrix_t(pack_f2h2(p0, p1));
       const uint32_t bv1 = movmatrix_t(pack_f2h2(p2, p3));
-      // P.V: A = V^T (rows channels, k = the 16 tokens) via ldmatrix.trans of the V rows
+      if (FP8) {
+        // P.V: A = V^T from ldmatrix.trans of the byte-pair blocks: a thread
+        // gets tokens 2c, 2c+1 (and 8 + 2c, 9 + 2c) of channels 2 g8 and
+        // 2 g8 + 1 of a chunk, which become the MMA rows g8 and g8 + 8 (the
+        // merge maps them back).  V past the sequence is zeroed in registers.
+        const uint32_t vb8 = smem_u32(raw + kUnit * 128);
+        const int lrow = (lane & 7) + 8 * (mi & 1);
+        const uint32_t mlo = (2 * c < valid_rows ? 0xffffu : 0u) | (2 * c + 1 < valid_rows ? 0xffff0000u : 0u);
+        const uint32_t mhi = (8 + 2 * c < valid_rows ? 0xffffu : 0u) | (9 + 2 * c < valid_rows ? 0xffff0000u : 0u);
 #pragma unroll
-      for (int mt = 0; mt < 8; ++mt) {
-        // matrices: (tokens 0-7, ch 16mt..+7), (tokens 0-7, ch +8..), (tokens 8-15, ch 16mt..), (8-15, +8)
-        const int vrow = (lane & 7) + 8 * (mi >> 1);
-        uint32_t a0, a1, a2, a3;
-        ldmatrix_x4_t(vb + off16(vrow, 2 * mt + (mi & 1)), a0, a1, a2, a3);
-        float o[4] = {0.f, 0.f, 0.f, 0.f};
-        mma_f16(o, a0, a1, a2, a3, bv0, bv1);
-        acc[mt][0] = fmaf(acc[mt][0], al0, o[0] * vs);
-        acc[mt][1] = fmaf(acc[mt][1], al1, o[1] * vs);
-        acc[mt][2] = fmaf(acc[mt][2], al0, o[2] * vs);
-        acc[mt][3] = fmaf(acc[mt][3], al1, o[3] * vs);
+        for (int mt = 0; mt < 8; mt += 2) {
+          uint32_t r0, r1, r2, r3;
+          ldmatrix_x4_t(vb8 + lrow * 128 + (((mt + (mi >> 1)) ^ (lrow & 7)) << 4), r0, r1, r2, r3);
+          const uint32_t rr[4] = {r0, r1, r2, r3};
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const uint32_t lo = rr[2 * h2], hi = rr[2 * h2 + 1];   // tokens 0-7, 8-15 of chunk mt + h2
+            float o[4] = {0.f, 0.f, 0.f, 0.f};
+            mma_f16(o, e4m3_bytes_to_f16x2(lo, 0x20) & mlo, e4m3_bytes_to_f16x2(lo, 0x31) & mlo,
+                    e4m3_bytes_to_f16x2(hi, 0x20) & mhi, e4m3_bytes_to_f16x2(hi, 0x31) & mhi, bv0, bv1);
+            float* ac = acc[mt + h2];
+            ac[0] = fmaf(ac[0], al0, o[0] * vs);
+            ac[1] = fmaf(ac[1], al1, o[1] * vs);
+            ac[2] = fmaf(ac[2], al0, o[2] * vs);
+            ac[3] = fmaf(ac[3], al1, o[3] * vs);
+          }
+        }
+      } else {
+        // P.V: A = V^T (rows channels, k = the 16 tokens) via ldmatrix.trans of the V rows
+        const uint32_t vb = smem_u32(raw + 2 * kHalf16);
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+          // matrices: (tokens 0-7, ch 16mt..+7), (tokens 0-7, ch +8..), (tokens 8-15, ch 16mt..), (8-15, +8)
+          const int vrow = (lane & 7) + 8 * (mi >> 1);
+          uint32_t a0, a1, a2, a3;
+          ldmatrix_x4_t(vb + off16(vrow, 2 * mt + (mi & 1)), a0, a1, a2, a3);
+          float o[4] = {0.f, 0.f, 0.f, 0.f};
+          mma_f16(o, a0, a1, a2, a3, bv0, bv1);
+          acc[mt][0] = fmaf(acc[mt][0], al0, o[0] * vs);
+          acc[mt][1] = fmaf(acc[mt][1], al1, o[1] * vs);
+          acc[mt][2] = fmaf(acc[mt][2], al0, o[2] * vs);
+          acc[mt][3] = fmaf(acc[mt][3], al1, o[3] * vs);
+        }
       }
     }
     __syncwarp();
@@ -271,7 +295,8 @@ __device__ void baseline_split(const BaselineArgs& p, const CUtensorMap* mk, con
   for (int mt = 0; mt < 8; ++mt)
 #pragma unroll
     for (int ri = 0; ri < 2; ++ri) {
-      const int d = 16 * mt + g8 + 8 * ri;
+      // MMA row g8 + 8 ri is channel 16 mt + g8 + 8 ri (fp16) or 16 mt + 2 g8 + ri (fp8)
+      const int d = FP8 ? 16 * mt + 2 * g8 + ri : 16 * mt + g8 + 8 * ri;
       aS[(warp * 8 + 2 * c) * kHeadDim + d] = acc[mt][2 * ri];
       aS[(warp * 8 + 2 * c + 1) * kHeadDim + d] = acc[mt][2 * ri + 1];
     }

@@ -1348,12 +1348,12 @@ cudaError_t noalloc_scratch(void** ptr, size_t* bytes) {
 }
 
 // Split-K geometry of the uncompressed baselines (baseline.cu).
-void decode_geometry(int B, int Hkv, int max_blocks, int* tiles_per_split, int* num_splits) {
+void decode_geometry(int B, int Hkv, int max_blocks, int ctas_per_sm, int* tiles_per_split, int* num_splits) {
   // Tiles per split T (a multiple of the 4 warps) chosen to minimise
-  // waves x (T / 4 tiles per warp + one tile of fixed cost), with about two
-  // resident CTAs per SM on a 148-SM part; ties go to the larger T.
+  // waves x (T / 4 tiles per warp + one tile of fixed cost), with
+  // ctas_per_sm resident CTAs per SM on a 148-SM part; ties go to the larger T.
   const long pairs = B * Hkv > 0 ? static_cast<long>(B) * Hkv : 1;
-  const long slots = 2 * 148;
+  const long slots = static_cast<long>(ctas_per_sm > 0 ? ctas_per_sm : 1) * 148;
   int best_t = kDWarps;
   double best = 1e300;
   for (int T = kDWarps; T <= 64; T += kDWarps) {

@@ -59,9 +59,14 @@ kvarn_status check_dims(const kvarn_decode_dims* dims, int max_group) {
 kvarn_status from_cuda(cudaError_t e) { return e == cudaSuccess ? KVARN_OK : KVARN_ERR_CUDA; }
 
 size_t partial_bytes(int B, int Hq, int Hkv, int max_blocks) {
-  int T = 0, ns = 0;
-  kvarn::decode_geometry(B, Hkv, max_blocks, &T, &ns);
-  return static_cast<size_t>(B) * Hq * (ns + 1) * kvarn::kPartialFloats * sizeof(float);
+  // room for the splits of either baseline's geometry
+  int ns_max = 0;
+  for (int fp8 = 0; fp8 < 2; ++fp8) {
+    int T = 0, ns = 0;
+    kvarn::decode_geometry(B, Hkv, max_blocks, kvarn::kBaselineCtasPerSm[fp8], &T, &ns);
+    ns_max = ns > ns_max ? ns : ns_max;
+  }
+  return static_cast<size_t>(B) * Hq * (ns_max + 1) * kvarn::kPartialFloats * sizeof(float);
 }
 
 // Uncompressed baselines: split-K partial records followed by B * Hkv int32
@@ -325,7 +330,8 @@ static kvarn_status baseline_impl(const void* q, const void* k_cache, const void
   p.G = dims->num_q_heads / dims->num_kv_heads;
   p.max_blocks = dims->max_blocks_per_seq;
   p.num_blocks = dims->num_blocks;
-  kvarn::decode_geometry(p.B, p.Hkv, p.max_blocks, &p.tiles_per_split, &p.num_splits);
+  kvarn::decode_geometry(p.B, p.Hkv, p.max_blocks, kvarn::kBaselineCtasPerSm[fp8 ? 1 : 0], &p.tiles_per_split,
+                         &p.num_splits);
   p.sm_scale = sm_scale > 0.f ? sm_scale : 1.0f / std::sqrt(static_cast<float>(KVARN_HEAD_DIM));
   p.k_scale = k_scale;
   p.v_scale = v_scale;

@@ -69,7 +69,11 @@ constexpr int kDecodeMaxCtas = 320;
 size_t decode_workspace(int B, int Hq, int Hkv, int qlen);
 
 // Split-K geometry of the uncompressed baselines: a pure function of the dims.
-void decode_geometry(int B, int Hkv, int max_blocks, int* tiles_per_split, int* num_splits);
+// Split geometry of the uncompressed baselines, for ctas_per_sm resident CTAs
+// per SM (kBaselineCtasPerSm[fp8]: the fp16 kernel's staging ring takes 128 KB
+// of shared memory, the e4m3 one 32 KB).
+void decode_geometry(int B, int Hkv, int max_blocks, int ctas_per_sm, int* tiles_per_split, int* num_splits);
+constexpr int kBaselineCtasPerSm[2] = {2, 4};
 
 cudaError_t launch_quantize(const QuantArgs& p, cudaStream_t stream);
 
