@@ -123,6 +123,33 @@ def test_baseline_argument_checks():
     assert r == 4
 
 
+def _baseline_splits(B, hkv, max_blocks, ctas_per_sm):
+    """The uncompressed baselines' split geometry restated: tiles per split T
+    (a multiple of 4) minimising waves x (T / 4 + 1) over ctas_per_sm x 148
+    slots, ties to the larger T; returns the number of splits."""
+    pairs, slots = max(1, B * hkv), ctas_per_sm * 148
+    best_t, best = 4, float("inf")
+    for t in range(4, 65, 4):
+        ns = -(-max_blocks // t)
+        cost = -(-(pairs * ns) // slots) * (t / 4 + 1)
+        if cost <= best:
+            best, best_t = cost, t
+        if ns == 1:
+            break
+    return max(1, -(-max_blocks // best_t))
+
+
+@pytest.mark.parametrize("B,hq,hkv,mb", [(8, 64, 8, 129), (16, 32, 8, 33), (4, 64, 8, 1025), (1, 8, 1, 1),
+                                         (2, 8, 2, 4), (64, 16, 2, 300)])
+def test_baseline_workspace_fits_both_geometries(B, hq, hkv, mb):
+    """The workspace holds the split records of the fp16 geometry (2 CTAs per
+    SM planned) and of the fp8 one (4), whichever is larger, then the B x Hkv
+    int32 arrival counters rounded to 16 bytes."""
+    ns = max(_baseline_splits(B, hkv, mb, 2), _baseline_splits(B, hkv, mb, 4))
+    counters = (B * hkv * 4 + 15) // 16 * 16
+    assert K.baseline_workspace_bytes(K.dims(B, hq, hkv, mb, 1024)) == B * hq * (ns + 1) * 528 + counters
+
+
 def test_binding_fails_loudly_without_library(tmp_path):
     """The binding refuses to import when libkvarn.so is absent (no fallback)."""
     import subprocess
