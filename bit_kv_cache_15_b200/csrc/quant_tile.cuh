@@ -146,11 +146,13 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
 }
 
 // The codes of a pair from their magic-add floats (1.5 * 2^23 + rne(y)): the
-// magic constant's low 16 bits are 0 and rne(y) lies in [0, 2^BITS - 1] (y is
-// (Z - zero) / step of the tile's own min and max, off by rounding errors far
-// below 1/2), so the low 16 bits of each float are its code and one byte
-// permute gives code.x | code.y << 16, ready to be shifted into its field of a
-// packed word (the fields do not overlap, so adding them is or-ing them).
+// magic constant's low 16 bits are 0 and rne(y) lies in [0, 2^BITS - 1], so
+// the low 16 bits of each float are its code and one byte permute gives
+// code.x | code.y << 16, ready to be shifted into its field of a packed word
+// (the fields do not overlap, so adding them is or-ing them).  y is
+// (Z - zero) / step for the tile's own min and max; its rounding error stays
+// far below 1/2 unless the tile's whole range is below fp32 resolution of its
+// offset (|zero / step| >= 2^23), where no fp32 grid can represent the tile.
 __device__ __forceinline__ uint32_t pair_codes(float2 r) {
   return __byte_perm(__float_as_uint(r.x), __float_as_uint(r.y), 0x5410);
 }
